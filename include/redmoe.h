@@ -1,0 +1,169 @@
+/*
+ * redmoe.h -- C ABI of libredmoe.so: one sparse mixture-of-experts FFN layer on an
+ * NVIDIA B200 (sm_100a), written for the Qwen3-Next-80B-A3B MoE block.
+ *
+ * The layer (shape from the "Architecture" page, section "Qwen3-Next shape": hidden
+ * 2048, 512 routed experts, top-10 per token, one shared expert, expert intermediate
+ * 512; the guide "DwarfStar Red Lite", section "What runs": every layer picks 10 of
+ * 512 experts) computes, for each token row x of [T, H]:
+ *
+ *   l[e] = x . Wr[e] (+ b[e])            router logits over E experts
+ *   ids  = the k largest logits, ordered by (logit desc, expert id asc)
+ *   w[j] = softmax(l)[ids_j] / sum_j' softmax(l)[ids_j']     renormalised weights
+ *   s    = sigmoid(x . g)                shared-expert gate
+ *   y_e  = Wd_e (silu(Wg_e x) * (Wu_e x)) SwiGLU expert, silu(a) = a sigmoid(a)
+ *   out  = sum_j w[j] y_{ids_j} + s y_shared
+ *
+ * The pages do not print this formula; it is the plainest reading of the shape facts
+ * (softmax gating with renormalised top-k weights, SwiGLU experts, a sigmoid-gated
+ * shared expert). Router, top-k and shared gate form one stage and the shared expert
+ * is one more expert slot, as in the DwarfStar Metal kernels ("Research notes, October
+ * 2026", section 1 "DwarfStar today").
+ *
+ * Conventions for every entry point:
+ *  - Every tensor pointer is DEVICE memory owned by the caller; the library allocates
+ *    no memory and keeps no state between calls except a per-device cache of device
+ *    attributes. Tensors are dense, row-major, contiguous.
+ *  - `stream` is a cudaStream_t (NULL: the legacy default stream). Work is only
+ *    enqueued; no call synchronises the host except redmoe_check_timeout().
+ *  - Arguments are validated on the host before anything is enqueued. On any error
+ *    status nothing has been enqueued and no output has been touched (except
+ *    REDMOE_ERR_CUDA, returned when a launch itself fails).
+ *  - Pointers to weights and activations must be 16-byte aligned; int4 scale tensors
+ *    2-byte aligned; id/count arrays 4-byte aligned.
+ *  - No entry point aborts or throws; all failures are status codes.
+ */
+#ifndef REDMOE_H
+#define REDMOE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define REDMOE_ABI_VERSION 1
+
+typedef enum {
+    REDMOE_OK = 0,
+    REDMOE_ERR_INVALID_ARG = 1,   /* null/misaligned pointer, bad size, bad enum value      */
+    REDMOE_ERR_UNSUPPORTED = 2,   /* valid arguments this build has no kernel for           */
+    REDMOE_ERR_WORKSPACE = 3,     /* workspace null or smaller than redmoe_workspace_bytes  */
+    REDMOE_ERR_CUDA = 4,          /* a CUDA runtime call or kernel launch failed            */
+    REDMOE_ERR_TIMEOUT = 5        /* a bounded in-kernel wait ran out (see check_timeout)   */
+} redmoe_status;
+
+/* Storage types. REDMOE_INT4G32 (expert weights only): a matrix [N, K] is stored as
+ * packed bytes [N, K/2] (element 2b in the low nibble of byte b, 2b+1 in the high
+ * nibble, nibble = code + 8, codes -8..7) plus bf16 scales [N, K/32], one per 32
+ * consecutive elements of a row; element value = scale * (nibble - 8). This format is
+ * defined by this library (the pages ship GGUF IQ types only). */
+typedef enum { REDMOE_F32 = 0, REDMOE_BF16 = 1, REDMOE_INT4G32 = 2 } redmoe_dtype;
+
+/* One MoE layer. All tensors device-resident, row-major; E = n_experts, H = hidden,
+ * I = inter, Is = shared_inter. The routed expert stacks keep the expert as the
+ * outer dimension, like the merged blk.N.ffn_{gate,up,down}_exps tensors of the
+ * "Red Lite v0.3 streaming development" page ("Implemented in dev1"). */
+typedef struct redmoe_layer {
+    int32_t hidden;          /* H, multiple of 64 (bf16/int4) or 32 (f32)                     */
+    int32_t n_experts;       /* E, 1..1024                                                    */
+    int32_t top_k;           /* k, 1..min(E, 32)                                              */
+    int32_t inter;           /* I, multiple of 64 (int4: 32; f32: 32)                         */
+    int32_t shared_inter;    /* Is, same rule as I                                            */
+    int32_t x_dtype;         /* redmoe_dtype of x: F32 or BF16                                */
+    int32_t router_dtype;    /* of router_w and shared_gate_w: F32 or BF16                    */
+    int32_t expert_dtype;    /* of all routed and shared expert weights                       */
+    const void *router_w;        /* [E, H]                                                    */
+    const float *router_bias;    /* [E] fp32 per-expert logit offset, or NULL                 */
+    const void *shared_gate_w;   /* [H]                                                       */
+    const void *w_gate;          /* [E, I, H]   (int4: u8 [E, I, H/2])                        */
+    const void *w_up;            /* [E, I, H]   (int4: u8 [E, I, H/2])                        */
+    const void *w_down;          /* [E, H, I]   (int4: u8 [E, H, I/2])                        */
+    const void *s_gate;          /* int4: bf16 [E, I, H/32]; otherwise NULL                   */
+    const void *s_up;            /* int4: bf16 [E, I, H/32]                                   */
+    const void *s_down;          /* int4: bf16 [E, H, I/32]                                   */
+    const void *sh_gate;         /* [Is, H]     (int4: u8 [Is, H/2])                          */
+    const void *sh_up;           /* [Is, H]                                                   */
+    const void *sh_down;         /* [H, Is]     (int4: u8 [H, Is/2])                          */
+    const void *sh_s_gate;       /* int4: bf16 [Is, H/32]; otherwise NULL                     */
+    const void *sh_s_up;         /* int4: bf16 [Is, H/32]                                     */
+    const void *sh_s_down;       /* int4: bf16 [H, Is/32]                                     */
+} redmoe_layer;
+
+/* Optional device outputs of the token->expert grouping (see redmoe_route_build). */
+typedef struct redmoe_route_debug {
+    int32_t *counts;    /* [E]      */
+    int32_t *offsets;   /* [E + 1]  */
+    int32_t *perm;      /* [T * k]  */
+} redmoe_route_debug;
+
+/* ABI version of the loaded library (REDMOE_ABI_VERSION it was built with). */
+int32_t redmoe_abi_version(void);
+
+/* Static, NUL-terminated description of a status code; never NULL. */
+const char *redmoe_status_string(int32_t status);
+
+/* Bytes of workspace redmoe_forward / redmoe_router / redmoe_route_build need for this
+ * layer at T tokens (a multiple of 256). Returns 0 if L is NULL or invalid or T < 0.
+ * The workspace is caller-owned device memory, 256-byte aligned. Its first 256 bytes
+ * are a control block that must be zero before the first use (redmoe_workspace_init
+ * or a memset); every call leaves it zero again, except one that ran into
+ * REDMOE_ERR_TIMEOUT, after which it must be re-initialised. Calls that share one
+ * workspace must be ordered on the GPU (same stream or synchronised streams). */
+size_t redmoe_workspace_bytes(const redmoe_layer *L, int32_t T);
+
+/* Zero the control block of a workspace on `stream` (an async memset of 256 bytes). */
+redmoe_status redmoe_workspace_init(void *workspace, size_t workspace_bytes, void *stream);
+
+/* The whole layer for T token rows.
+ *   x        [T, H] in L->x_dtype
+ *   out      [T, H] fp32, overwritten (not accumulated)
+ *   topk_ids [T, k] int32, expert ids ordered by logit descending, ties to the lower id
+ *   topk_w   [T, k] fp32, renormalised weights in the same order (sum to 1 per row)
+ *   dbg      NULL, or device arrays that receive the token->expert grouping
+ * T == 0 is a valid empty call: nothing is enqueued. Decode sizes (T <= 4) run one
+ * persistent kernel; larger T runs the batched (grouped-GEMM) path, which needs bf16
+ * x, router and experts (other dtypes at T > 4 return REDMOE_ERR_UNSUPPORTED). */
+redmoe_status redmoe_forward(const redmoe_layer *L, const void *x, int32_t T, float *out,
+                             int32_t *topk_ids, float *topk_w, void *workspace,
+                             size_t workspace_bytes, const redmoe_route_debug *dbg, void *stream);
+
+/* The router stage alone: logits, top-k ids, renormalised weights, shared gate.
+ *   topk_ids [T, k] int32, topk_w [T, k] fp32, shared_gate [T] fp32 = sigmoid(x . g),
+ *   logits [T, E] fp32 (router_bias included) or NULL. */
+redmoe_status redmoe_router(const redmoe_layer *L, const void *x, int32_t T, int32_t *topk_ids,
+                            float *topk_w, float *shared_gate, float *logits, void *workspace,
+                            size_t workspace_bytes, void *stream);
+
+/* Token->expert grouping of a [T, k] id matrix (k distinct ids per row, each in
+ * [0, E)): counts[e] = rows routed to e; offsets[0] = 0, offsets[e+1] = offsets[e] +
+ * counts[e]; perm[offsets[e] + r] = t*k + j for the r-th row (t, j) routed to e in
+ * increasing t. Bit-exact and deterministic. The batched path of redmoe_forward uses
+ * the same kernel. Out-of-range ids are not detected on the device: they are skipped
+ * and the outputs are then unspecified. Workspace: redmoe_workspace_bytes of any layer
+ * with these E and k at this T (or at least 256 bytes + 4*(E+1)*ceil(T/64) bytes). */
+redmoe_status redmoe_route_build(const int32_t *topk_ids, int32_t T, int32_t k, int32_t E,
+                                 int32_t *counts, int32_t *offsets, int32_t *perm,
+                                 void *workspace, size_t workspace_bytes, void *stream);
+
+/* n_layers independent layers of the same shape and dtypes, one after the other on
+ * `stream` (layer l reads xs[l] and writes outs[l], ids[l], ws[l]; each array holds
+ * n_layers device pointers and lives in HOST memory). Equivalent to n_layers calls of
+ * redmoe_forward; the decode sizes (T <= 4) run them in one persistent launch, which
+ * lets the L2 prefetch of layer l+1's router and shared-expert weights overlap layer l. */
+redmoe_status redmoe_forward_stack(const redmoe_layer *layers, int32_t n_layers,
+                                   const void *const *xs, int32_t T, float *const *outs,
+                                   int32_t *const *ids, float *const *ws, void *workspace,
+                                   size_t workspace_bytes, void *stream);
+
+/* Synchronise `stream`, then read the workspace's error word: REDMOE_ERR_TIMEOUT if an
+ * in-kernel grid barrier gave up waiting (bounded at about one second) since the last
+ * redmoe_workspace_init, else REDMOE_OK. REDMOE_ERR_CUDA if the stream reports an error. */
+redmoe_status redmoe_check_timeout(const void *workspace, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* REDMOE_H */

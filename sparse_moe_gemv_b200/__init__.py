@@ -1,0 +1,216 @@
+"""Python binding of libredmoe.so (C ABI: include/redmoe.h).
+
+Argument marshalling only: every step of the layer runs in the library's CUDA kernels.
+torch provides device memory and streams. The binding never computes a result itself
+and has no fallback: if the library is missing it raises.
+
+Names match the C entry points (redmoe_forward, redmoe_router, redmoe_route_build,
+redmoe_forward_stack, redmoe_workspace_bytes, redmoe_workspace_init,
+redmoe_check_timeout, redmoe_status_string, redmoe_abi_version).
+"""
+
+from __future__ import annotations
+
+import ctypes as C
+import os
+import threading
+from typing import Dict, Optional, Sequence
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libredmoe.so")
+ABI_VERSION = 1
+DTYPES = {"f32": 0, "bf16": 1, "int4g32": 2}
+STATUS = {0: "REDMOE_OK", 1: "REDMOE_ERR_INVALID_ARG", 2: "REDMOE_ERR_UNSUPPORTED", 3: "REDMOE_ERR_WORKSPACE",
+          4: "REDMOE_ERR_CUDA", 5: "REDMOE_ERR_TIMEOUT"}
+# entry points declared in include/redmoe.h
+SYMBOLS = ("redmoe_abi_version", "redmoe_status_string", "redmoe_workspace_bytes", "redmoe_workspace_init",
+           "redmoe_forward", "redmoe_router", "redmoe_route_build", "redmoe_forward_stack",
+           "redmoe_check_timeout")
+
+_lock = threading.Lock()
+_lib = None
+
+
+class RedmoeError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = int(status)
+        super().__init__(f"{where}: {STATUS.get(self.status, self.status)} ({redmoe_status_string(self.status)})")
+
+
+class _Layer(C.Structure):
+    _fields_ = [
+        ("hidden", C.c_int32), ("n_experts", C.c_int32), ("top_k", C.c_int32), ("inter", C.c_int32),
+        ("shared_inter", C.c_int32), ("x_dtype", C.c_int32), ("router_dtype", C.c_int32),
+        ("expert_dtype", C.c_int32),
+        ("router_w", C.c_void_p), ("router_bias", C.c_void_p), ("shared_gate_w", C.c_void_p),
+        ("w_gate", C.c_void_p), ("w_up", C.c_void_p), ("w_down", C.c_void_p),
+        ("s_gate", C.c_void_p), ("s_up", C.c_void_p), ("s_down", C.c_void_p),
+        ("sh_gate", C.c_void_p), ("sh_up", C.c_void_p), ("sh_down", C.c_void_p),
+        ("sh_s_gate", C.c_void_p), ("sh_s_up", C.c_void_p), ("sh_s_down", C.c_void_p),
+    ]
+
+
+class _RouteDebug(C.Structure):
+    _fields_ = [("counts", C.c_void_p), ("offsets", C.c_void_p), ("perm", C.c_void_p)]
+
+
+def load():
+    """Load libredmoe.so (built in-tree). Raises if it has not been built."""
+    global _lib
+    with _lock:
+        if _lib is not None:
+            return _lib
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with `python -m sparse_moe_gemv_b200.build`")
+        lib = C.CDLL(LIB_PATH)
+        P, i32, sz = C.c_void_p, C.c_int32, C.c_size_t
+        lib.redmoe_abi_version.restype = i32
+        lib.redmoe_abi_version.argtypes = []
+        lib.redmoe_status_string.restype = C.c_char_p
+        lib.redmoe_status_string.argtypes = [i32]
+        lib.redmoe_workspace_bytes.restype = sz
+        lib.redmoe_workspace_bytes.argtypes = [P, i32]
+        lib.redmoe_workspace_init.restype = i32
+        lib.redmoe_workspace_init.argtypes = [P, sz, P]
+        lib.redmoe_forward.restype = i32
+        lib.redmoe_forward.argtypes = [P, P, i32, P, P, P, P, sz, P, P]
+        lib.redmoe_router.restype = i32
+        lib.redmoe_router.argtypes = [P, P, i32, P, P, P, P, P, sz, P]
+        lib.redmoe_route_build.restype = i32
+        lib.redmoe_route_build.argtypes = [P, i32, i32, i32, P, P, P, P, sz, P]
+        lib.redmoe_forward_stack.restype = i32
+        lib.redmoe_forward_stack.argtypes = [P, i32, P, i32, P, P, P, P, sz, P]
+        lib.redmoe_check_timeout.restype = i32
+        lib.redmoe_check_timeout.argtypes = [P, P]
+        if lib.redmoe_abi_version() != ABI_VERSION:
+            raise RuntimeError("libredmoe.so ABI version mismatch")
+        _lib = lib
+        return lib
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else t.data_ptr()
+
+
+def _stream(stream) -> Optional[int]:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, torch.cuda.Stream):
+        return stream.cuda_stream
+    return int(stream)
+
+
+def _check(status: int, where: str):
+    if status != 0:
+        raise RedmoeError(status, where)
+
+
+class Layer:
+    """A layer's device tensors plus its C descriptor.
+
+    `tensors` uses the names of the C struct (router_w, router_bias, shared_gate_w,
+    w_gate, w_up, w_down, s_gate, s_up, s_down, sh_gate, sh_up, sh_down, sh_s_gate,
+    sh_s_up, sh_s_down); the tensors are kept alive by this object.
+    """
+
+    def __init__(self, tensors: Dict[str, Optional[torch.Tensor]], hidden: int, n_experts: int, top_k: int,
+                 inter: int, shared_inter: int, x_dtype: str = "bf16", router_dtype: str = "bf16",
+                 expert_dtype: str = "bf16"):
+        self.tensors = dict(tensors)
+        s = _Layer()
+        s.hidden, s.n_experts, s.top_k, s.inter, s.shared_inter = hidden, n_experts, top_k, inter, shared_inter
+        s.x_dtype, s.router_dtype, s.expert_dtype = DTYPES[x_dtype], DTYPES[router_dtype], DTYPES[expert_dtype]
+        for name, _ in _Layer._fields_[8:]:
+            setattr(s, name, _ptr(self.tensors.get(name)))
+        self.struct = s
+        self.hidden, self.n_experts, self.top_k = hidden, n_experts, top_k
+        self.inter, self.shared_inter = inter, shared_inter
+        self.x_dtype, self.router_dtype, self.expert_dtype = x_dtype, router_dtype, expert_dtype
+
+    @classmethod
+    def from_shape(cls, tensors, shape):
+        """`shape` has attributes H, E, k, I, Is, x_dtype, router_dtype, expert_dtype."""
+        return cls(tensors, shape.H, shape.E, shape.k, shape.I, shape.Is, shape.x_dtype, shape.router_dtype,
+                   shape.expert_dtype)
+
+    @property
+    def ref(self):
+        return C.byref(self.struct)
+
+
+def redmoe_abi_version() -> int:
+    return int(load().redmoe_abi_version())
+
+
+def redmoe_status_string(status: int) -> str:
+    return load().redmoe_status_string(int(status)).decode()
+
+
+def redmoe_workspace_bytes(layer: Layer, T: int) -> int:
+    return int(load().redmoe_workspace_bytes(layer.ref, int(T)))
+
+
+def redmoe_workspace_init(workspace: torch.Tensor, stream=None) -> None:
+    _check(load().redmoe_workspace_init(_ptr(workspace), workspace.numel() * workspace.element_size(),
+                                        _stream(stream)), "redmoe_workspace_init")
+
+
+def new_workspace(layer: Layer, T: int, device=None) -> torch.Tensor:
+    """A zeroed workspace tensor of redmoe_workspace_bytes(layer, T) bytes."""
+    n = redmoe_workspace_bytes(layer, T)
+    if n == 0:
+        raise ValueError("invalid layer or token count")
+    return torch.zeros(n, dtype=torch.uint8, device=device or "cuda")
+
+
+def redmoe_forward(layer: Layer, x: torch.Tensor, out: torch.Tensor, topk_ids: torch.Tensor, topk_w: torch.Tensor,
+                   workspace: torch.Tensor, dbg: Optional[Sequence[torch.Tensor]] = None, stream=None,
+                   T: Optional[int] = None) -> None:
+    """out[T,H] fp32, topk_ids[T,k] int32, topk_w[T,k] fp32 <- layer(x[T,H])."""
+    lib = load()
+    dbg_s = None
+    if dbg is not None:
+        dbg_s = _RouteDebug(_ptr(dbg[0]), _ptr(dbg[1]), _ptr(dbg[2]))
+    T = x.shape[0] if T is None else T
+    st = lib.redmoe_forward(layer.ref, _ptr(x), int(T), _ptr(out), _ptr(topk_ids), _ptr(topk_w),
+                            _ptr(workspace), workspace.numel() * workspace.element_size(),
+                            None if dbg_s is None else C.byref(dbg_s), _stream(stream))
+    _check(st, "redmoe_forward")
+
+
+def redmoe_router(layer: Layer, x: torch.Tensor, topk_ids: torch.Tensor, topk_w: torch.Tensor,
+                  shared_gate: torch.Tensor, workspace: torch.Tensor, logits: Optional[torch.Tensor] = None,
+                  stream=None) -> None:
+    st = load().redmoe_router(layer.ref, _ptr(x), int(x.shape[0]), _ptr(topk_ids), _ptr(topk_w), _ptr(shared_gate),
+                              _ptr(logits), _ptr(workspace), workspace.numel() * workspace.element_size(),
+                              _stream(stream))
+    _check(st, "redmoe_router")
+
+
+def redmoe_route_build(topk_ids: torch.Tensor, n_experts: int, counts: torch.Tensor, offsets: torch.Tensor,
+                       perm: torch.Tensor, stream=None) -> None:
+    T, k = topk_ids.shape
+    st = load().redmoe_route_build(_ptr(topk_ids), int(T), int(k), int(n_experts), _ptr(counts), _ptr(offsets),
+                                   _ptr(perm), None, 0, _stream(stream))
+    _check(st, "redmoe_route_build")
+
+
+def redmoe_forward_stack(layers: Sequence[Layer], xs: Sequence[torch.Tensor], outs: Sequence[torch.Tensor],
+                         ids: Sequence[torch.Tensor], ws: Sequence[torch.Tensor], workspace: torch.Tensor,
+                         stream=None) -> None:
+    n = len(layers)
+    arr = (_Layer * n)(*[l.struct for l in layers])
+    P = C.c_void_p * n
+    T = xs[0].shape[0] if n else 0
+    st = load().redmoe_forward_stack(C.cast(arr, C.c_void_p), n, C.cast(P(*[_ptr(t) for t in xs]), C.c_void_p),
+                                     int(T), C.cast(P(*[_ptr(t) for t in outs]), C.c_void_p),
+                                     C.cast(P(*[_ptr(t) for t in ids]), C.c_void_p),
+                                     C.cast(P(*[_ptr(t) for t in ws]), C.c_void_p), _ptr(workspace),
+                                     workspace.numel() * workspace.element_size(), _stream(stream))
+    _check(st, "redmoe_forward_stack")
+
+
+def redmoe_check_timeout(workspace: torch.Tensor, stream=None) -> None:
+    _check(load().redmoe_check_timeout(_ptr(workspace), _stream(stream)), "redmoe_check_timeout")

@@ -1,0 +1,136 @@
+// Device helpers shared by the redmoe kernels (sm_100a).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace redmoe {
+
+enum : int { DT_F32 = 0, DT_BF16 = 1, DT_INT4 = 2 };
+
+// Bits of the workspace error word.
+enum : int { ERRBIT_TIMEOUT = 1 };
+
+constexpr unsigned FULL = 0xffffffffu;
+
+// Control block at the start of every workspace (256 bytes, zero between calls).
+struct Control {
+    unsigned bar_count;   // grid-barrier arrivals of the current barrier
+    unsigned bar_gen;     // grid-barrier generation (only ever increases)
+    int err;              // ERRBIT_* set by any kernel that gave up waiting
+    unsigned pad[61];
+};
+static_assert(sizeof(Control) == 256, "control block is 256 bytes");
+
+// ----------------------------------------------------------------- conversions
+__device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+__device__ __forceinline__ float bf16f(uint16_t b) { return __uint_as_float(uint32_t(b) << 16); }
+
+// Round-to-nearest-even fp32 -> bf16 bits (inputs are finite).
+__device__ __forceinline__ uint16_t f2bf(float f) {
+    uint32_t u = __float_as_uint(f);
+    u += 0x7fffu + ((u >> 16) & 1u);
+    return uint16_t(u >> 16);
+}
+
+// Order-preserving map of a float onto uint32 (larger float -> larger key); -0 == +0.
+__device__ __forceinline__ uint32_t order_key(float f) {
+    if (f == 0.0f) f = 0.0f;
+    uint32_t u = __float_as_uint(f);
+    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+__device__ __forceinline__ float key_to_float(uint32_t k) {
+    uint32_t u = (k & 0x80000000u) ? (k & 0x7fffffffu) : ~k;
+    return __uint_as_float(u);
+}
+
+// ------------------------------------------------------------------- loads
+// Streaming read-only 16-byte load: weights are read once per call, keep them out of L1.
+__device__ __forceinline__ uint4 ld_stream(const void* p) {
+    uint4 v;
+    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(p));
+    return v;
+}
+__device__ __forceinline__ uint16_t ld_stream_u16(const void* p) {
+    uint16_t v;
+    asm volatile("ld.global.nc.L1::no_allocate.u16 %0, [%1];" : "=h"(v) : "l"(p));
+    return v;
+}
+
+// L2 prefetch of the 16-byte-aligned part of [p, p + bytes): the start is rounded up
+// and the end down, so the prefetched range never leaves the buffer.
+__device__ __forceinline__ void prefetch_l2(const void* p, uint64_t bytes) {
+    const uint64_t a = reinterpret_cast<uint64_t>(p);
+    const uint64_t s = (a + 15u) & ~uint64_t(15);
+    const uint64_t e = (a + bytes) & ~uint64_t(15);
+    for (uint64_t q = s; q < e; q += (1u << 20)) {
+        const uint32_t n = uint32_t((e - q) < (1u << 20) ? (e - q) : (1u << 20));
+        asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" :: "l"(q), "r"(n) : "memory");
+    }
+}
+
+__device__ __forceinline__ uint64_t globaltimer_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+__device__ __forceinline__ unsigned ld_acquire_gpu(const unsigned* p) {
+    unsigned v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+__device__ __forceinline__ void st_release_gpu(unsigned* p, unsigned v) {
+    asm volatile("st.release.gpu.global.u32 [%0], %1;" :: "l"(p), "r"(v) : "memory");
+}
+__device__ __forceinline__ int ld_relaxed_gpu(const int* p) {
+    int v;
+    asm volatile("ld.relaxed.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+// ------------------------------------------------------------- warp reductions
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(FULL, v, o);
+    return v;
+}
+
+// ------------------------------------------------------------ grid barrier
+// Barrier across all blocks of a cooperative launch (every block is resident, so every
+// block eventually arrives). The wait is bounded: after `timeout_ns` (or once another
+// block has recorded a timeout) the block records ERRBIT_TIMEOUT and continues, so a
+// fault in the barrier can never hang the GPU; the host reads the error word.
+// Uses a self-resetting arrival counter plus a generation word.
+__device__ __forceinline__ void grid_barrier(Control* ctl, unsigned nblocks, uint64_t timeout_ns) {
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        const unsigned gen = ld_acquire_gpu(&ctl->bar_gen);
+        __threadfence();
+        const unsigned arrived = atomicAdd(&ctl->bar_count, 1u);
+        if (arrived == nblocks - 1) {
+            atomicExch(&ctl->bar_count, 0u);
+            __threadfence();
+            st_release_gpu(&ctl->bar_gen, gen + 1u);
+        } else {
+            const uint64_t t0 = globaltimer_ns();
+            uint32_t spins = 0;
+            while (ld_acquire_gpu(&ctl->bar_gen) == gen) {
+                if ((++spins & 255u) == 0u) {
+                    if (ld_relaxed_gpu(&ctl->err) != 0 || globaltimer_ns() - t0 > timeout_ns ||
+                        spins > (1u << 26)) {
+                        atomicOr(&ctl->err, ERRBIT_TIMEOUT);
+                        break;
+                    }
+                }
+                __nanosleep(32);
+            }
+        }
+        __threadfence();
+    }
+    __syncthreads();
+}
+
+}  // namespace redmoe

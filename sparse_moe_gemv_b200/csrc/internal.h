@@ -1,0 +1,60 @@
+// Declarations shared between the .cu files of libredmoe (not part of the C ABI).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "../../include/redmoe.h"
+
+namespace redmoe {
+
+constexpr int DECODE_MAX_T = 4;        // decode kernel handles 1..4 token rows
+constexpr int MAX_TOPK = 32;
+constexpr int MAX_EXPERTS = 1024;
+constexpr int MAX_STACK = 64;          // layers per persistent decode launch
+constexpr uint64_t BARRIER_TIMEOUT_NS = 1000000000ull;  // 1 s
+
+inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+// One layer as the decode kernel sees it (pointers into caller memory).
+struct DecLayer {
+    const void* router_w;
+    const float* router_bias;
+    const void* shared_gate_w;
+    const void* w_gate;
+    const void* w_up;
+    const void* w_down;
+    const uint16_t* s_gate;
+    const uint16_t* s_up;
+    const uint16_t* s_down;
+    const void* sh_gate;
+    const void* sh_up;
+    const void* sh_down;
+    const uint16_t* sh_s_gate;
+    const uint16_t* sh_s_up;
+    const uint16_t* sh_s_down;
+    const void* x;
+    float* out;
+    int32_t* ids;
+    float* w;
+};
+
+// Workspace carve-up of the decode path (byte offsets from the workspace base).
+struct DecodeWs {
+    size_t logits, sgate, hsh, hrt, total;
+};
+DecodeWs decode_ws_layout(int T, int E, int k, int I, int Is);
+
+// Launch the persistent decode kernel over n_layers layers (1..MAX_STACK).
+redmoe_status launch_decode(const redmoe_layer* shape, const DecLayer* layers, int n_layers, int T,
+                            void* workspace, cudaStream_t stream, int* launches);
+
+// Device attributes cached per device.
+struct DevInfo {
+    int sm_count;
+    int max_smem_optin;
+};
+bool get_dev_info(DevInfo* out);
+
+}  // namespace redmoe

@@ -1,0 +1,110 @@
+// Router stage for any number of token rows (the batched path and redmoe_router):
+//   router_logits_kernel  l[t, e] = x_t . Wr[e] (+ b[e])   (CUDA cores, rows streamed once
+//                         per block of 4 tokens; the prefill path computes the same logits
+//                         with the tensor-core GEMM instead)
+//   topk_kernel           per token (one warp): top-k of the logits with ties to the lower
+//                         id, renormalised weights, shared gate sigmoid(x . g), and
+//                         optionally a zeroed output row for the scatter-add combine.
+// Router, top-k and shared gate belong to one stage of the layer ("Research notes,
+// October 2026", section 1 "DwarfStar today": router, top-k and shared gate run in one
+// kernel); here the logits of a large batch come from a GEMM, so the top-k and gate
+// run as the epilogue kernel that follows it.
+#include "common.cuh"
+#include "gemv.cuh"
+#include "internal.h"
+#include "topk.cuh"
+
+namespace redmoe {
+
+namespace {
+
+constexpr int RL_THREADS = 256;
+constexpr int RL_WARPS = RL_THREADS / 32;
+constexpr int RL_TOK = 4;  // tokens per block
+
+template <int XT, int RT>
+__global__ void __launch_bounds__(RL_THREADS) router_logits_kernel(const void* x, int T, int H, int E,
+                                                                   const void* wr, const float* bias,
+                                                                   float* logits) {
+    extern __shared__ __align__(128) unsigned char smem[];
+    uint4* xs = reinterpret_cast<uint4*>(smem);
+    const int xstride = staged_bytes(H, RT, XT) / 16;
+    const int t0 = blockIdx.y * RL_TOK;
+    const int nt = min(RL_TOK, T - t0);
+    for (int t = 0; t < nt; ++t)
+        stage_vec<RT, XT>(xs + t * xstride, static_cast<const char*>(x) + size_t(t0 + t) * H * vbytes(XT), H, false);
+    __syncthreads();
+    const int lane = threadIdx.x & 31;
+    const int e = blockIdx.x * RL_WARPS + (threadIdx.x >> 5);
+    if (e >= E) return;
+    float acc[RL_TOK] = {0.f, 0.f, 0.f, 0.f};
+    row_dots<RT, XT>(static_cast<const char*>(wr) + size_t(e) * row_bytes(RT, H), nullptr, H, xs, xstride, nt, lane, acc);
+    const float b = bias ? bias[e] : 0.0f;
+#pragma unroll
+    for (int t = 0; t < RL_TOK; ++t) {
+        const float v = warp_sum(acc[t]);
+        if (lane == 0 && t < nt) logits[size_t(t0 + t) * E + e] = v + b;
+    }
+}
+
+template <int XT, int RT>
+__global__ void __launch_bounds__(RL_THREADS) topk_kernel(const float* logits, int T, int E, int k, const void* x,
+                                                          const void* g, int H, int32_t* ids, float* w,
+                                                          float* sgate, float* zero_out) {
+    const int lane = threadIdx.x & 31;
+    const int t = blockIdx.x * RL_WARPS + (threadIdx.x >> 5);
+    if (t >= T) return;
+    warp_topk(logits + size_t(t) * E, E, k, ids + size_t(t) * k, w + size_t(t) * k);
+    float acc = 0.0f;
+    for (int h = lane; h < H; h += 32) {
+        float xv, gv;
+        if constexpr (XT == DT_BF16) xv = bf16f(static_cast<const uint16_t*>(x)[size_t(t) * H + h]);
+        else xv = static_cast<const float*>(x)[size_t(t) * H + h];
+        if constexpr (RT == DT_BF16) gv = bf16f(static_cast<const uint16_t*>(g)[h]);
+        else gv = static_cast<const float*>(g)[h];
+        acc = fmaf(xv, gv, acc);
+    }
+    acc = warp_sum(acc);
+    if (lane == 0 && sgate) sgate[t] = 1.0f / (1.0f + expf(-acc));
+    if (zero_out) {
+        float4* o = reinterpret_cast<float4*>(zero_out + size_t(t) * H);
+        for (int i = lane; i < H / 4; i += 32) o[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+}
+
+template <int XT, int RT>
+redmoe_status launch_router_dt(const redmoe_layer* L, const void* x, int T, float* logits, int32_t* ids,
+                               float* w, float* sgate, float* zero_out, bool compute_logits,
+                               cudaStream_t stream, int* launches) {
+    const int H = L->hidden, E = L->n_experts;
+    if (compute_logits) {
+        const int smem = RL_TOK * staged_bytes(H, RT, XT);
+        auto kern = router_logits_kernel<XT, RT>;
+        if (smem > 48 * 1024 &&
+            cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+            return REDMOE_ERR_CUDA;
+        dim3 grid((E + RL_WARPS - 1) / RL_WARPS, (T + RL_TOK - 1) / RL_TOK);
+        kern<<<grid, RL_THREADS, smem, stream>>>(x, T, H, E, L->router_w, L->router_bias, logits);
+        if (cudaGetLastError() != cudaSuccess) return REDMOE_ERR_CUDA;
+        if (launches) *launches += 1;
+    }
+    topk_kernel<XT, RT><<<(T + RL_WARPS - 1) / RL_WARPS, RL_THREADS, 0, stream>>>(
+        logits, T, E, L->top_k, x, L->shared_gate_w, H, ids, w, sgate, zero_out);
+    if (cudaGetLastError() != cudaSuccess) return REDMOE_ERR_CUDA;
+    if (launches) *launches += 1;
+    return REDMOE_OK;
+}
+
+}  // namespace
+
+redmoe_status launch_router(const redmoe_layer* L, const void* x, int T, float* logits, int32_t* ids, float* w,
+                            float* sgate, float* zero_out, bool compute_logits, cudaStream_t stream,
+                            int* launches) {
+    if (L->x_dtype == DT_F32 && L->router_dtype == DT_F32)
+        return launch_router_dt<DT_F32, DT_F32>(L, x, T, logits, ids, w, sgate, zero_out, compute_logits, stream, launches);
+    if (L->x_dtype == DT_BF16 && L->router_dtype == DT_BF16)
+        return launch_router_dt<DT_BF16, DT_BF16>(L, x, T, logits, ids, w, sgate, zero_out, compute_logits, stream, launches);
+    return REDMOE_ERR_UNSUPPORTED;
+}
+
+}  // namespace redmoe
