@@ -1,0 +1,480 @@
+"""MoE-layer benchmark on B200 (one process per GPU).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl redmoe|reference]
+
+Workloads (synthetic seeded layers of the Qwen3-Next-80B-A3B MoE shape: hidden 2048,
+512 experts, top-10, expert and shared intermediate 512):
+
+  decode_t1   (default) one token through one bf16 layer per step; the steps rotate over
+              12 distinct layers (38.7 GB), so no step finds its weights in L2
+  fewrow_t2 / fewrow_t3   a 12-layer bf16 stack of independent layers, 2 or 3 tokens
+  int4_48     a 48-layer int4 group-32 stack, one token
+  prefill     a 2048-token chunk through one bf16 layer with Zipf(1.1) router offsets
+
+One JSON line on rank 0: the device-timed throughput (CUDA events on the launching
+stream, graph replay of the steps, barrier + synchronize around the timed region, max
+over ranks), the roofline of the dominant kernel, the end-to-end figure through the C
+ABI with pinned host buffers, the fp64 oracle on the host cores, and the SM clocks seen
+during the timed region. The path does not shard (one layer fits one GPU): with N > 1
+every rank runs its own replica ("replicas only"), the value is the sum over ranks.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+import moe_inputs as mi  # noqa: E402
+
+METRIC = "MoE-layer tokens/s at 1 B200; decode HBM GB/s (% of peak); prefill TFLOP/s"
+FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
+QWEN = mi.LayerShape(H=2048, E=512, k=10, I=512, Is=512)
+QWEN_INT4 = mi.LayerShape(H=2048, E=512, k=10, I=512, Is=512, expert_dtype="int4g32")
+
+WORKLOADS = {
+    "decode_t1": dict(shape=QWEN, T=1, layers=12, stack=False, seed=1000, kernel="decode_kernel",
+                      desc="Qwen3-Next-shaped MoE layer, bf16 weights / fp32 accumulate, decode T=1"),
+    "fewrow_t2": dict(shape=QWEN, T=2, layers=12, stack=True, seed=2000, kernel="decode_kernel",
+                      desc="12 distinct Qwen3-Next-shaped bf16 layers back to back, T=2"),
+    "fewrow_t3": dict(shape=QWEN, T=3, layers=12, stack=True, seed=2000, kernel="decode_kernel",
+                      desc="12 distinct Qwen3-Next-shaped bf16 layers back to back, T=3"),
+    "int4_48": dict(shape=QWEN_INT4, T=1, layers=48, stack=True, seed=4000, kernel="decode_kernel",
+                    desc="48 distinct Qwen3-Next-shaped layers, int4 group-32 experts, decode T=1"),
+}
+
+
+# ------------------------------------------------------------------ helpers
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return float(d["hbm_gbs"]), float(d["bf16_tflops"]), float(d.get("bf16_tflops_sustained", 0)), "measured"
+    return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, 1400.0, "fallback"
+
+
+def expert_bytes(shape):
+    """Bytes of one expert's three matrices (int4: packed codes + bf16 scales)."""
+    H, I = shape.H, shape.I
+    if shape.expert_dtype == "int4g32":
+        return 3 * (H * I // 2 + H * I // 32 * 2)
+    return 3 * H * I * (4 if shape.expert_dtype == "f32" else 2)
+
+
+def shared_bytes(shape):
+    H, I = shape.H, shape.Is
+    if shape.expert_dtype == "int4g32":
+        return 3 * (H * I // 2 + H * I // 32 * 2)
+    return 3 * H * I * (4 if shape.expert_dtype == "f32" else 2)
+
+
+def layer_call_bytes(shape, T, distinct):
+    """Algorithmic HBM bytes of one layer call: every weight the math needs read once
+    (router, shared gate, the distinct routed experts, the shared expert), x read once,
+    out / ids / weights written once."""
+    rb = 4 if shape.router_dtype == "f32" else 2
+    xb = 4 if shape.x_dtype == "f32" else 2
+    return (shape.E * shape.H * rb + shape.H * rb + distinct * expert_bytes(shape) + shared_bytes(shape)
+            + T * shape.H * xb + T * shape.H * 4 + T * shape.k * 8)
+
+
+def source_digest(kernel_file):
+    h = hashlib.sha256()
+    for f in sorted(os.listdir(os.path.join(ROOT, "sparse_moe_gemv_b200", "csrc"))):
+        if f.endswith((".cu", ".cuh", ".h")):
+            h.update(open(os.path.join(ROOT, "sparse_moe_gemv_b200", "csrc", f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def profile_traffic(workload):
+    """DRAM bytes per launch from the committed ncu summary, if it matches this source."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    d = json.load(open(p)).get(workload)
+    if not d or d.get("source_digest") != source_digest(None):
+        return None
+    return d.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML while the timed region runs."""
+
+    REASONS = {
+        "gpu_idle": 0x1, "applications_clocks_setting": 0x2, "sw_power_cap": 0x4, "hw_slowdown": 0x8,
+        "sync_boost": 0x10, "sw_thermal_slowdown": 0x20, "hw_thermal_slowdown": 0x40,
+        "hw_power_brake_slowdown": 0x80, "display_clock_setting": 0x100,
+    }
+
+    def __init__(self, device_index):
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self._stop = threading.Event()
+        self._thread = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        except Exception:  # NVML missing: report no clocks rather than fail the run
+            self.nv = None
+
+    def _run(self):
+        while not self._stop.is_set():
+            self._sample()
+            time.sleep(0.005)
+
+    def _sample(self):
+        try:
+            self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+            r = self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+            for name, bit in self.REASONS.items():
+                if r & bit and name != "gpu_idle":
+                    self.reasons.add(name)
+        except Exception:
+            pass
+
+    def __enter__(self):
+        if self.nv is not None:
+            self._sample()
+            self._thread = threading.Thread(target=self._run, daemon=True)
+            self._thread.start()
+        return self
+
+    def __exit__(self, *a):
+        if self._thread is not None:
+            self._stop.set()
+            self._thread.join()
+            self._sample()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0}
+        return {"sm_mhz": float(statistics.median(self.samples)), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+# ---------------------------------------------------------------- distributed
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(local)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        torch.distributed.barrier()
+
+
+def max_over_ranks(v, world):
+    if world == 1:
+        return v
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def sum_over_ranks(v, world):
+    if world == 1:
+        return v
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.SUM)
+    return float(t.item())
+
+
+# ------------------------------------------------------------- CPU baseline
+def cpu_oracle_sample(wl, seconds=10.0):
+    """The fp64 oracle on the host cores over a bounded sample of the workload: decode
+    tokens through layer 0 of the workload (one oracle call, OpenMP over tokens)."""
+    import oracle
+    shape = wl["shape"]
+    cores = oracle.num_threads()
+    L = mi.make_layer(shape, wl["seed"], "cuda")
+    lay = mi.layer_to_numpy(L)
+    del L
+    x1 = mi.to_numpy(mi.make_x(shape, 1, wl["seed"] + 99, "cpu"))
+    t0 = time.perf_counter()
+    oracle.forward(lay, shape, x1)
+    t1 = time.perf_counter() - t0
+    n = int(max(cores, min(4096, seconds * cores / max(t1, 1e-3))))
+    n = max(cores, (n // cores) * cores)
+    x = mi.to_numpy(mi.make_x(shape, n, wl["seed"] + 123, "cpu"))
+    t0 = time.perf_counter()
+    oracle.forward(lay, shape, x)
+    el = time.perf_counter() - t0
+    return {"value": n / el, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+            "sample": f"{n} decode tokens through one {wl['desc']} layer, one oracle call "
+                      f"(fp64, OpenMP over tokens), {el:.1f} s wall"}
+
+
+def reference_arm(args, wl, world, rank):
+    """The fp64 oracle as the reference implementation, timed on the host cores."""
+    import oracle
+    if rank != 0:
+        return None
+    shape = wl["shape"]
+    T = wl["T"]
+    cores = oracle.num_threads()
+    nl = min(wl["layers"], 2)
+    layers = []
+    for l in range(nl):
+        L = mi.make_layer(shape, wl["seed"] + l, "cuda")
+        layers.append(mi.layer_to_numpy(L))
+        del L
+    torch.cuda.empty_cache()
+    xs = [mi.to_numpy(mi.make_x(shape, T, wl["seed"] + 7 * s, "cpu")) for s in range(4)]
+    tokens_per_step = T * (wl["layers"] if wl["stack"] else 1)
+
+    def step(s):
+        for l in range(wl["layers"] if wl["stack"] else 1):
+            oracle.forward(layers[(s + l) % nl], shape, xs[s % 4])
+
+    for s in range(args.warmup):
+        step(s)
+    budget = 120.0
+    t0 = time.perf_counter()
+    done = 0
+    for s in range(args.steps):
+        step(s)
+        done += 1
+        if time.perf_counter() - t0 > budget:
+            break
+    el = time.perf_counter() - t0
+    value = done * tokens_per_step / el
+    unit = "tokens/s"
+    sample = (f"{done} of {args.steps} steps (time-bounded at {budget:.0f} s), each "
+              f"{'a ' + str(wl['layers']) + '-layer stack' if wl['stack'] else 'one layer'} at T={T}, "
+              f"fp64 oracle, {cores} threads")
+    return {"metric": METRIC, "value": value, "unit": unit, "n_gpus": 1, "steps": done, "warmup": args.warmup,
+            "ms_per_step": 1e3 * el / max(done, 1), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": wl["desc"], "tokens_per_step": tokens_per_step, "parallelism": "replicas"},
+            "impl": "reference",
+            "cpu_baseline": {"value": value, "unit": unit, "cores": cores, "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+# ------------------------------------------------------------------ GPU arm
+def build_workload(wl, smg):
+    shape, T, nl = wl["shape"], wl["T"], wl["layers"]
+    tens = [mi.make_layer(shape, wl["seed"] + l, "cuda") for l in range(nl)]
+    lays = [smg.Layer.from_shape(t, shape) for t in tens]
+    xs = [mi.make_x(shape, T, wl["seed"] + l, "cuda") for l in range(nl)]
+    outs = [torch.empty(T, shape.H, device="cuda") for _ in range(nl)]
+    ids = [torch.empty(T, shape.k, dtype=torch.int32, device="cuda") for _ in range(nl)]
+    ws_ = [torch.empty(T, shape.k, device="cuda") for _ in range(nl)]
+    work = smg.new_workspace(lays[0], T)
+    return dict(tens=tens, lays=lays, xs=xs, outs=outs, ids=ids, ws=ws_, work=work)
+
+
+def make_step(wl, smg, B, stream):
+    """step(i): the i-th step's launches on `stream`."""
+    nl = wl["layers"]
+    if wl["stack"]:
+        def step(i):
+            smg.redmoe_forward_stack(B["lays"], B["xs"], B["outs"], B["ids"], B["ws"], B["work"], stream=stream)
+        return step, 1 if nl <= 64 else math.ceil(nl / 64)
+
+    def step(i):
+        l = i % nl
+        smg.redmoe_forward(B["lays"][l], B["xs"][l], B["outs"][l], B["ids"][l], B["ws"][l], B["work"], stream=stream)
+    return step, 1
+
+
+def capture(step, n, stream):
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        for i in range(n):
+            step(i)
+    return g
+
+
+def gpu_arm(args, wl, world, rank, local):
+    import sparse_moe_gemv_b200 as smg
+    smg.load()
+    shape, T = wl["shape"], wl["T"]
+    B = build_workload(wl, smg)
+    stream = torch.cuda.Stream()
+    step, launches_per_step = make_step(wl, smg, B, stream)
+    torch.cuda.synchronize()
+    # graphs: one rotation of the layers per replay (stack workloads: one stack per replay)
+    chunk = 1 if wl["stack"] else wl["layers"]
+    graph = capture(step, chunk, stream)
+    K, W = args.steps, args.warmup
+    torch.cuda.synchronize()
+
+    def run(nsteps):
+        full, rem = divmod(nsteps, chunk)
+        for _ in range(full):
+            graph.replay()
+        for i in range(rem):
+            step(i)
+
+    with torch.cuda.stream(stream):
+        run(W)
+    torch.cuda.synchronize()
+    smg.redmoe_check_timeout(B["work"], stream=stream)
+
+    ev0 = torch.cuda.Event(enable_timing=True)
+    ev1 = torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        with torch.cuda.stream(stream):
+            ev0.record(stream)
+            run(K)
+            ev1.record(stream)
+        torch.cuda.synchronize()
+    barrier(world)
+    smg.redmoe_check_timeout(B["work"], stream=stream)
+    el_ms = ev0.elapsed_time(ev1)
+    el_ms = max_over_ranks(el_ms, world)
+    tokens_per_step = T * (wl["layers"] if wl["stack"] else 1)
+    value = sum_over_ranks(K * tokens_per_step, world) / (el_ms / 1e3)
+
+    # distinct experts per layer call, from the ids of the last step of each layer
+    distinct = []
+    for l in range(wl["layers"]):
+        distinct.append(len(set(B["ids"][l].view(-1).tolist())))
+    layers_per_step = wl["layers"] if wl["stack"] else 1
+    if wl["stack"]:
+        bytes_per_launch = sum(layer_call_bytes(shape, T, d) for d in distinct)
+    else:
+        bytes_per_launch = sum(layer_call_bytes(shape, T, d) for d in distinct) / len(distinct)
+    launches = K * launches_per_step
+    launch_s = el_ms / 1e3 / launches
+    hbm, bf16, bf16_sus, src = peaks()
+    achieved = bytes_per_launch / launch_s / 1e9
+
+    # end to end through the C ABI with pinned host buffers: per step H2D x, forward, D2H out/ids/w
+    e2e = e2e_arm(args, wl, smg, B, stream, world)
+    result = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K, "warmup": W,
+        "ms_per_step": el_ms / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16" if shape.expert_dtype == "bf16" else ("int4g32" if shape.expert_dtype == "int4g32" else "f32"),
+        "data": "synthetic",
+        "config": {"workload": wl["desc"], "tokens_per_step": tokens_per_step, "layers_in_rotation": wl["layers"],
+                   "l2": "inputs larger than L2: each step reads a different layer's weights "
+                         f"({wl['layers']} distinct layers)" if not wl["stack"] else
+                         f"inputs larger than L2: {wl['layers']} distinct layers per step",
+                   "parallelism": "replicas" if world > 1 else "single GPU", "timing": "CUDA graph replay"},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
+                     "traffic": profile_traffic(args.workload), "kernel": wl["kernel"],
+                     "bytes_per_launch": bytes_per_launch, "launch_us": launch_s * 1e6,
+                     "peak_source": f"{src} (MEASURED_PEAKS.json hbm_gbs)" if src == "measured" else "fallback"},
+        "e2e": e2e,
+        "gpu_launches": launches,
+        "clocks": clk.summary(),
+    }
+    return result
+
+
+def e2e_arm(args, wl, smg, B, stream, world):
+    shape, T = wl["shape"], wl["T"]
+    nl = wl["layers"]
+    K = args.steps
+    xb = 4 if shape.x_dtype == "f32" else 2
+    xdt = torch.float32 if shape.x_dtype == "f32" else torch.bfloat16
+    hx = [B["xs"][l].cpu().pin_memory() for l in range(nl)]
+    hout = torch.empty(T, shape.H, dtype=torch.float32).pin_memory()
+    hids = torch.empty(T, shape.k, dtype=torch.int32).pin_memory()
+    hw = torch.empty(T, shape.k, dtype=torch.float32).pin_memory()
+    dx = [torch.empty(T, shape.H, dtype=xdt, device="cuda") for _ in range(nl)]
+
+    def step(i):
+        if wl["stack"]:
+            for l in range(nl):
+                dx[l].copy_(hx[l], non_blocking=True)
+            smg.redmoe_forward_stack(B["lays"], dx, B["outs"], B["ids"], B["ws"], B["work"], stream=stream)
+            for l in range(nl):
+                hout.copy_(B["outs"][l], non_blocking=True)
+                hids.copy_(B["ids"][l], non_blocking=True)
+                hw.copy_(B["ws"][l], non_blocking=True)
+        else:
+            l = i % nl
+            dx[l].copy_(hx[l], non_blocking=True)
+            smg.redmoe_forward(B["lays"][l], dx[l], B["outs"][l], B["ids"][l], B["ws"][l], B["work"], stream=stream)
+            hout.copy_(B["outs"][l], non_blocking=True)
+            hids.copy_(B["ids"][l], non_blocking=True)
+            hw.copy_(B["ws"][l], non_blocking=True)
+
+    n_e2e = K
+    with torch.cuda.stream(stream):
+        for i in range(min(args.warmup, 50)):
+            step(i)
+    torch.cuda.synchronize()
+    barrier(world)
+    t0 = time.perf_counter()
+    with torch.cuda.stream(stream):
+        for i in range(n_e2e):
+            step(i)
+    stream.synchronize()
+    el = time.perf_counter() - t0
+    el = max_over_ranks(el, world)
+    per = (nl if wl["stack"] else 1)
+    tokens = n_e2e * T * per
+    h2d = T * shape.H * xb * per
+    d2h = (T * shape.H * 4 + T * shape.k * 8) * per
+    return {"value": sum_over_ranks(tokens, world) / el, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h, "steps": n_e2e,
+            "how": "redmoe_forward through the C ABI per step; pinned host x copied in, out/ids/w copied out, "
+                   "host wall clock around the K steps"}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20000)
+    ap.add_argument("--warmup", type=int, default=240)
+    ap.add_argument("--workload", default="decode_t1", choices=sorted(WORKLOADS))
+    ap.add_argument("--impl", default="redmoe", choices=["redmoe", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--layers", type=int, default=None,
+                    help="override the number of distinct layers (small cases for profiler captures)")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    wl = dict(WORKLOADS[args.workload])
+    if args.layers:
+        wl["layers"] = args.layers
+    world, rank, local = dist_setup()
+    if args.impl == "reference":
+        res = reference_arm(args, wl, world, rank)
+        if rank == 0:
+            print(json.dumps(res), flush=True)
+        if world > 1:
+            torch.distributed.destroy_process_group()
+        return
+    res = gpu_arm(args, wl, world, rank, local)
+    if rank == 0:
+        if world == 1 and not args.no_cpu_baseline:
+            res["cpu_baseline"] = cpu_oracle_sample(wl)
+        print(json.dumps(res), flush=True)
+    if world > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

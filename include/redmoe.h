@@ -80,7 +80,7 @@ typedef struct redmoe_layer {
     const void *w_gate;          /* [E, I, H]   (int4: u8 [E, I, H/2])                        */
     const void *w_up;            /* [E, I, H]   (int4: u8 [E, I, H/2])                        */
     const void *w_down;          /* [E, H, I]   (int4: u8 [E, H, I/2])                        */
-    const void *s_gate;          /* int4: bf16 [E, I, H/32]; otherwise NULL                   */
+    const void *s_gate;          /* int4: bf16 [E, I, H/32], 16-byte aligned; otherwise NULL  */
     const void *s_up;            /* int4: bf16 [E, I, H/32]                                   */
     const void *s_down;          /* int4: bf16 [E, H, I/32]                                   */
     const void *sh_gate;         /* [Is, H]     (int4: u8 [Is, H/2])                          */

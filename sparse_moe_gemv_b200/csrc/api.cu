@@ -68,7 +68,7 @@ redmoe_status check_layer(const redmoe_layer* L) {
     const void* sc[] = {L->s_gate, L->s_up, L->s_down, L->sh_s_gate, L->sh_s_up, L->sh_s_down};
     for (const void* p : sc) {
         if (wt == DT_INT4) {
-            if (!p || !aligned(p, 2)) return REDMOE_ERR_INVALID_ARG;
+            if (!p || !aligned(p, 16)) return REDMOE_ERR_INVALID_ARG;
         }
     }
     return REDMOE_OK;

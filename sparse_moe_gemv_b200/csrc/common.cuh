@@ -15,8 +15,8 @@ constexpr unsigned FULL = 0xffffffffu;
 
 // Control block at the start of every workspace (256 bytes, zero between calls).
 struct Control {
-    unsigned bar_count;   // grid-barrier arrivals of the current barrier
-    unsigned bar_gen;     // grid-barrier generation (only ever increases)
+    unsigned bar_count;   // grid-barrier arrivals since the launch began
+    unsigned bar_gen;     // blocks that have finished the launch (grid_exit)
     int err;              // ERRBIT_* set by any kernel that gave up waiting
     unsigned pad[61];
 };
@@ -91,6 +91,60 @@ __device__ __forceinline__ int ld_relaxed_gpu(const int* p) {
     return v;
 }
 
+// ------------------------------------------------------- mbarrier / bulk copies
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" :: "r"(smem_u32(bar)), "r"(count) : "memory");
+}
+// Make mbarrier initialisation visible to the async proxy (bulk copies, tensor cores).
+__device__ __forceinline__ void fence_mbar_init() {
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+// Order this thread's generic-proxy shared-memory accesses before later async-proxy ones.
+__device__ __forceinline__ void fence_proxy_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+// Order earlier generic-proxy global writes (seen through a grid barrier) before this
+// thread's later async-proxy (bulk copy) reads of global memory.
+__device__ __forceinline__ void fence_proxy_async_global() {
+    asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" :: "r"(smem_u32(bar)), "r"(bytes)
+                 : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}"
+        : "=r"(ok) : "r"(smem_u32(bar)), "r"(parity) : "memory");
+    return ok != 0;
+}
+// Bounded wait for the phase of `bar` with the given parity. Gives up after timeout_ns
+// (or at once if another thread has already recorded a timeout): sets ERRBIT_TIMEOUT in
+// *err and returns false; the caller carries on with whatever the buffer holds.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* err, uint64_t timeout_ns) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = globaltimer_ns();
+    for (uint32_t i = 1;; ++i) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if ((i & 63u) == 0u) {
+            if (ld_relaxed_gpu(err) != 0 || globaltimer_ns() - t0 > timeout_ns || i > (1u << 26)) {
+                atomicOr(err, ERRBIT_TIMEOUT);
+                return false;
+            }
+        }
+    }
+}
+// 1-D bulk copy global -> shared (this CTA), completion counted on `bar` in bytes.
+// dst and src 16-byte aligned, bytes a multiple of 16.
+__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+                 :: "r"(smem_u32(dst)), "l"(src), "r"(bytes), "r"(smem_u32(bar)) : "memory");
+}
+
 // ------------------------------------------------------------- warp reductions
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
@@ -100,37 +154,73 @@ __device__ __forceinline__ float warp_sum(float v) {
 
 // ------------------------------------------------------------ grid barrier
 // Barrier across all blocks of a cooperative launch (every block is resident, so every
-// block eventually arrives). The wait is bounded: after `timeout_ns` (or once another
-// block has recorded a timeout) the block records ERRBIT_TIMEOUT and continues, so a
-// fault in the barrier can never hang the GPU; the host reads the error word.
-// Uses a self-resetting arrival counter plus a generation word.
-__device__ __forceinline__ void grid_barrier(Control* ctl, unsigned nblocks, uint64_t timeout_ns) {
+// block eventually arrives). Barrier number b of a launch waits until the arrival counter
+// reaches (b + 1) * nblocks; arrivals are fire-and-forget reductions. grid_exit() must end
+// the launch: its last block resets the counter for the next launch. The wait is bounded:
+// after `timeout_ns` (or once another block has recorded a timeout) the block records
+// ERRBIT_TIMEOUT and continues, so a fault can never hang the GPU; the host reads the
+// error word.
+__device__ __forceinline__ void grid_barrier(Control* ctl, unsigned nblocks, unsigned index, uint64_t timeout_ns) {
     __syncthreads();
     if (threadIdx.x == 0) {
-        const unsigned gen = ld_acquire_gpu(&ctl->bar_gen);
         __threadfence();
-        const unsigned arrived = atomicAdd(&ctl->bar_count, 1u);
-        if (arrived == nblocks - 1) {
-            atomicExch(&ctl->bar_count, 0u);
-            __threadfence();
-            st_release_gpu(&ctl->bar_gen, gen + 1u);
-        } else {
+        asm volatile("red.relaxed.gpu.global.add.u32 [%0], 1;" :: "l"(&ctl->bar_count) : "memory");
+        const unsigned target = (index + 1u) * nblocks;
+        if (ld_acquire_gpu(&ctl->bar_count) < target) {
             const uint64_t t0 = globaltimer_ns();
-            uint32_t spins = 0;
-            while (ld_acquire_gpu(&ctl->bar_gen) == gen) {
-                if ((++spins & 255u) == 0u) {
-                    if (ld_relaxed_gpu(&ctl->err) != 0 || globaltimer_ns() - t0 > timeout_ns ||
-                        spins > (1u << 26)) {
+            for (uint32_t spins = 1; ld_acquire_gpu(&ctl->bar_count) < target; ++spins) {
+                if ((spins & 63u) == 0u) {
+                    if (ld_relaxed_gpu(&ctl->err) != 0 || globaltimer_ns() - t0 > timeout_ns || spins > (1u << 26)) {
                         atomicOr(&ctl->err, ERRBIT_TIMEOUT);
                         break;
                     }
                 }
-                __nanosleep(32);
             }
         }
         __threadfence();
     }
     __syncthreads();
+}
+
+// The two halves of grid_barrier, for work that may overlap the wait (arrive, then do
+// independent work, then wait). Same bounded wait and error reporting.
+__device__ __forceinline__ void grid_arrive(Control* ctl) {
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        __threadfence();
+        asm volatile("red.relaxed.gpu.global.add.u32 [%0], 1;" :: "l"(&ctl->bar_count) : "memory");
+    }
+}
+__device__ __forceinline__ void grid_wait(Control* ctl, unsigned nblocks, unsigned index, uint64_t timeout_ns) {
+    if (threadIdx.x == 0) {
+        const unsigned target = (index + 1u) * nblocks;
+        if (ld_acquire_gpu(&ctl->bar_count) < target) {
+            const uint64_t t0 = globaltimer_ns();
+            for (uint32_t spins = 1; ld_acquire_gpu(&ctl->bar_count) < target; ++spins) {
+                if ((spins & 63u) == 0u) {
+                    if (ld_relaxed_gpu(&ctl->err) != 0 || globaltimer_ns() - t0 > timeout_ns || spins > (1u << 26)) {
+                        atomicOr(&ctl->err, ERRBIT_TIMEOUT);
+                        break;
+                    }
+                }
+            }
+        }
+        __threadfence();
+    }
+    __syncthreads();
+}
+
+// End of a launch that used grid_barrier: the last block out resets the counters.
+__device__ __forceinline__ void grid_exit(Control* ctl, unsigned nblocks) {
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        __threadfence();
+        const unsigned done = atomicAdd(&ctl->bar_gen, 1u);
+        if (done == nblocks - 1u) {
+            atomicExch(&ctl->bar_count, 0u);
+            atomicExch(&ctl->bar_gen, 0u);
+        }
+    }
 }
 
 }  // namespace redmoe

@@ -4,14 +4,13 @@
 // 32 int4); lane L of a warp reads chunks L, L + 32, ... so that one warp instruction
 // moves 512 contiguous bytes. The activation vectors the row is dotted with live in
 // shared memory in a chunk-interleaved layout (see stage_vec) so that the matching
-// activation reads are conflict-free for every weight type.
+// activation reads are conflict-free for every weight type. Products accumulate in
+// fp32 (packed f32x2 fused multiply-adds, two partial sums per lane).
 #pragma once
 
 #include "common.cuh"
 
 namespace redmoe {
-
-constexpr int GEMV_G = 8;   // 16-byte chunks per lane per row group (loads in flight)
 
 template <int W> struct Wv;
 template <> struct Wv<DT_F32> { static constexpr int V = 4; };
@@ -37,8 +36,9 @@ __host__ __device__ inline int staged_bytes(int K, int w, int vt) {
 
 // ------------------------------------------------------------------ staging
 // Copy a K-vector (bf16 or f32 in global memory) into the chunk-interleaved layout for
-// weight type W. `coherent` selects L2-only loads for data written earlier in this
-// launch by other blocks.
+// weight type W: the P 16-byte pieces of the activations matching weight chunk c sit at
+// slots ((c / 32) * P + q) * 32 + c % 32. `coherent` selects L2-only loads for data
+// written earlier in this launch by other blocks.
 template <int W, int VT>
 __device__ void stage_vec(uint4* dst, const void* src, int K, bool coherent) {
     constexpr int V = Wv<W>::V;
@@ -61,47 +61,64 @@ __device__ void stage_vec(uint4* dst, const void* src, int K, bool coherent) {
     }
 }
 
-// --------------------------------------------------------------- chunk dot
-// Dot of one 16-byte weight chunk (iteration ii, lane position L) with its staged
-// activations. int4: returns sum (nibble - 8) * x; the caller applies the group scale.
-__device__ __forceinline__ float nib(uint32_t w, int n) {
-    return __uint_as_float(0x4B000000u | ((w >> (4 * n)) & 15u)) - 8388616.0f;
+// --------------------------------------------------------------- f32x2 math
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
+    float2 d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;"
+        : "=l"(reinterpret_cast<uint64_t&>(d))
+        : "l"(reinterpret_cast<const uint64_t&>(a)), "l"(reinterpret_cast<const uint64_t&>(b)),
+          "l"(reinterpret_cast<const uint64_t&>(c)));
+    return d;
+}
+__device__ __forceinline__ float2 fadd2(float2 a, float2 b) {
+    float2 d;
+    asm("add.f32x2 %0, %1, %2;"
+        : "=l"(reinterpret_cast<uint64_t&>(d))
+        : "l"(reinterpret_cast<const uint64_t&>(a)), "l"(reinterpret_cast<const uint64_t&>(b)));
+    return d;
+}
+__device__ __forceinline__ float2 bf2(uint32_t w) { return make_float2(bf16lo(w), bf16hi(w)); }
+__device__ __forceinline__ float2 f2(uint32_t a, uint32_t b) { return make_float2(__uint_as_float(a), __uint_as_float(b)); }
+// int4 nibbles n and n+1 of w as floats (nibble - 8): exponent-trick conversion, exact.
+__device__ __forceinline__ float2 nib2(uint32_t w, int n) {
+    const float2 m = make_float2(__uint_as_float(0x4B000000u | ((w >> (4 * n)) & 15u)),
+                                 __uint_as_float(0x4B000000u | ((w >> (4 * n + 4)) & 15u)));
+    return fadd2(m, make_float2(-8388616.0f, -8388616.0f));
 }
 
+// --------------------------------------------------------------- chunk dot
+// Accumulate the dot of one 16-byte weight chunk (iteration ii, lane position L) with its
+// staged activations into acc (two partial sums). int4: acc gets sum (nibble - 8) * x; the
+// caller applies the group scale.
 template <int W, int VT>
-__device__ __forceinline__ float chunk_dot(const uint4& w, const uint4* xs, int ii, int L) {
+__device__ __forceinline__ float2 chunk_dot(const uint4& w, const uint4* xs, int ii, int L, float2 acc) {
     constexpr int P = Pc<W, VT>::P;
     const uint4* b = xs + ii * P * 32 + L;
-    float acc = 0.0f;
     if constexpr (W == DT_BF16 && VT == DT_BF16) {
         const uint4 x = b[0];
-        acc = fmaf(bf16lo(w.x), bf16lo(x.x), acc); acc = fmaf(bf16hi(w.x), bf16hi(x.x), acc);
-        acc = fmaf(bf16lo(w.y), bf16lo(x.y), acc); acc = fmaf(bf16hi(w.y), bf16hi(x.y), acc);
-        acc = fmaf(bf16lo(w.z), bf16lo(x.z), acc); acc = fmaf(bf16hi(w.z), bf16hi(x.z), acc);
-        acc = fmaf(bf16lo(w.w), bf16lo(x.w), acc); acc = fmaf(bf16hi(w.w), bf16hi(x.w), acc);
+        acc = ffma2(bf2(w.x), bf2(x.x), acc);
+        acc = ffma2(bf2(w.y), bf2(x.y), acc);
+        acc = ffma2(bf2(w.z), bf2(x.z), acc);
+        acc = ffma2(bf2(w.w), bf2(x.w), acc);
     } else if constexpr (W == DT_BF16 && VT == DT_F32) {
         const uint4 x0 = b[0], x1 = b[32];
-        acc = fmaf(bf16lo(w.x), __uint_as_float(x0.x), acc); acc = fmaf(bf16hi(w.x), __uint_as_float(x0.y), acc);
-        acc = fmaf(bf16lo(w.y), __uint_as_float(x0.z), acc); acc = fmaf(bf16hi(w.y), __uint_as_float(x0.w), acc);
-        acc = fmaf(bf16lo(w.z), __uint_as_float(x1.x), acc); acc = fmaf(bf16hi(w.z), __uint_as_float(x1.y), acc);
-        acc = fmaf(bf16lo(w.w), __uint_as_float(x1.z), acc); acc = fmaf(bf16hi(w.w), __uint_as_float(x1.w), acc);
+        acc = ffma2(bf2(w.x), f2(x0.x, x0.y), acc);
+        acc = ffma2(bf2(w.y), f2(x0.z, x0.w), acc);
+        acc = ffma2(bf2(w.z), f2(x1.x, x1.y), acc);
+        acc = ffma2(bf2(w.w), f2(x1.z, x1.w), acc);
     } else if constexpr (W == DT_F32 && VT == DT_F32) {
         const uint4 x = b[0];
-        acc = fmaf(__uint_as_float(w.x), __uint_as_float(x.x), acc);
-        acc = fmaf(__uint_as_float(w.y), __uint_as_float(x.y), acc);
-        acc = fmaf(__uint_as_float(w.z), __uint_as_float(x.z), acc);
-        acc = fmaf(__uint_as_float(w.w), __uint_as_float(x.w), acc);
+        acc = ffma2(f2(w.x, w.y), f2(x.x, x.y), acc);
+        acc = ffma2(f2(w.z, w.w), f2(x.z, x.w), acc);
     } else if constexpr (W == DT_INT4 && VT == DT_BF16) {
         const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
             const uint4 x = b[q * 32];
-            const uint32_t xw[4] = {x.x, x.y, x.z, x.w};
-#pragma unroll
-            for (int m = 0; m < 4; ++m) {
-                acc = fmaf(nib(ws[q], 2 * m), bf16lo(xw[m]), acc);
-                acc = fmaf(nib(ws[q], 2 * m + 1), bf16hi(xw[m]), acc);
-            }
+            acc = ffma2(nib2(ws[q], 0), bf2(x.x), acc);
+            acc = ffma2(nib2(ws[q], 2), bf2(x.y), acc);
+            acc = ffma2(nib2(ws[q], 4), bf2(x.z), acc);
+            acc = ffma2(nib2(ws[q], 6), bf2(x.w), acc);
         }
     } else if constexpr (W == DT_INT4 && VT == DT_F32) {
         const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
@@ -110,85 +127,97 @@ __device__ __forceinline__ float chunk_dot(const uint4& w, const uint4* xs, int 
             const uint4 x = b[p * 32];
             const uint32_t wq = ws[p >> 1];
             const int n0 = (p & 1) * 4;
-            acc = fmaf(nib(wq, n0 + 0), __uint_as_float(x.x), acc);
-            acc = fmaf(nib(wq, n0 + 1), __uint_as_float(x.y), acc);
-            acc = fmaf(nib(wq, n0 + 2), __uint_as_float(x.z), acc);
-            acc = fmaf(nib(wq, n0 + 3), __uint_as_float(x.w), acc);
+            acc = ffma2(nib2(wq, n0), f2(x.x, x.y), acc);
+            acc = ffma2(nib2(wq, n0 + 2), f2(x.z, x.w), acc);
         }
     }
     return acc;
 }
 
-// Lane-partial dots of one weight row (K elements, type W) with T staged vectors
-// (vector t at xs + t * xstride uint4s). Row groups of G chunks per lane are loaded
-// before use so that each lane has G 16-byte loads in flight.
-template <int W, int VT, int NT>
-__device__ __forceinline__ void row_dots(const void* row, const uint16_t* srow, int K, const uint4* xs,
-                                         int xstride, int T, int lane, float (&acc)[NT]) {
-    const int nch = K / Wv<W>::V;
-    const int nit = (nch + 31) / 32;
+// Scaled accumulation: acc += s * (chunk . x) for int4, acc += chunk . x otherwise.
+template <int W, int VT>
+__device__ __forceinline__ float2 chunk_dot_s(const uint4& w, float s, const uint4* xs, int ii, int L, float2 acc) {
+    if constexpr (W == DT_INT4) {
+        const float2 d = chunk_dot<W, VT>(w, xs, ii, L, make_float2(0.f, 0.f));
+        return ffma2(make_float2(s, s), d, acc);
+    } else {
+        (void)s;
+        return chunk_dot<W, VT>(w, xs, ii, L, acc);
+    }
+}
+
+// Weighted accumulation: acc += s * (chunk . x) for every weight type (s carries the
+// int4 group scale times a routing weight, or just the routing weight).
+template <int W, int VT>
+__device__ __forceinline__ float2 chunk_dot_w(const uint4& w, float s, const uint4* xs, int ii, int L, float2 acc) {
+    const float2 d = chunk_dot<W, VT>(w, xs, ii, L, make_float2(0.f, 0.f));
+    return ffma2(make_float2(s, s), d, acc);
+}
+
+// 16-byte chunks per lane loaded before use in a row job (loads in flight per lane)
+template <int W> struct RowGroup { static constexpr int G = (W == DT_BF16) ? 8 : 2; };
+
+// Lane-partial dots of one weight row (nch 16-byte chunks) with the T staged vectors
+// (vector t at xs + t * xstride uint4s).
+template <int W, int VT, int T>
+__device__ __forceinline__ void row_dots(const void* row, const uint16_t* srow, int nch, const uint4* xs,
+                                         int xstride, int lane, float2 (&acc)[T]) {
+    constexpr int G = RowGroup<W>::G;
+    const int nit = (nch + 31) >> 5;
     const uint4* r = static_cast<const uint4*>(row);
-    for (int g0 = 0; g0 < nit; g0 += GEMV_G) {
-        uint4 wc[GEMV_G];
-        float sc[GEMV_G];
+    for (int g0 = 0; g0 < nit; g0 += G) {
+        uint4 wc[G];
+        float sc[G];
 #pragma unroll
-        for (int i = 0; i < GEMV_G; ++i) {
+        for (int i = 0; i < G; ++i) {
             const int c = (g0 + i) * 32 + lane;
             const bool ok = (g0 + i < nit) && c < nch;
             wc[i] = ok ? ld_stream(r + c) : make_uint4(0u, 0u, 0u, 0u);
+            sc[i] = 0.0f;
             if constexpr (W == DT_INT4) sc[i] = ok ? bf16f(ld_stream_u16(srow + c)) : 0.0f;
         }
 #pragma unroll
-        for (int i = 0; i < GEMV_G; ++i) {
+        for (int i = 0; i < G; ++i) {
             if (g0 + i < nit) {
 #pragma unroll
-                for (int t = 0; t < NT; ++t) {
-                    if (t < T) {
-                        float d = chunk_dot<W, VT>(wc[i], xs + t * xstride, g0 + i, lane);
-                        if constexpr (W == DT_INT4) d *= sc[i];
-                        acc[t] += d;
-                    }
-                }
+                for (int t = 0; t < T; ++t)
+                    acc[t] = chunk_dot_s<W, VT>(wc[i], sc[i], xs + t * xstride, g0 + i, lane, acc[t]);
             }
         }
     }
 }
 
-// Gate and up rows of one expert row index together (both K = H), then SwiGLU.
-template <int W, int VT, int NT>
-__device__ __forceinline__ void pair_dots(const void* grow, const uint16_t* gs, const void* urow,
-                                          const uint16_t* us, int K, const uint4* xs, int xstride,
-                                          int T, int lane, float (&a)[NT], float (&u)[NT]) {
-    const int nch = K / Wv<W>::V;
-    const int nit = (nch + 31) / 32;
+// Gate and up rows of one expert row index together (both K = H).
+template <int W, int VT, int T>
+__device__ __forceinline__ void pair_dots(const void* grow, const uint16_t* gs, const void* urow, const uint16_t* us,
+                                          int nch, const uint4* xs, int xstride, int lane, float2 (&a)[T],
+                                          float2 (&u)[T]) {
+    constexpr int G = RowGroup<W>::G;
+    const int nit = (nch + 31) >> 5;
     const uint4* gr = static_cast<const uint4*>(grow);
     const uint4* ur = static_cast<const uint4*>(urow);
-    for (int g0 = 0; g0 < nit; g0 += GEMV_G) {
-        uint4 wg[GEMV_G], wu[GEMV_G];
-        float sg[GEMV_G], su[GEMV_G];
+    for (int g0 = 0; g0 < nit; g0 += G) {
+        uint4 wg[G], wu[G];
+        float sg[G], su[G];
 #pragma unroll
-        for (int i = 0; i < GEMV_G; ++i) {
+        for (int i = 0; i < G; ++i) {
             const int c = (g0 + i) * 32 + lane;
             const bool ok = (g0 + i < nit) && c < nch;
             wg[i] = ok ? ld_stream(gr + c) : make_uint4(0u, 0u, 0u, 0u);
             wu[i] = ok ? ld_stream(ur + c) : make_uint4(0u, 0u, 0u, 0u);
+            sg[i] = su[i] = 0.0f;
             if constexpr (W == DT_INT4) {
                 sg[i] = ok ? bf16f(ld_stream_u16(gs + c)) : 0.0f;
                 su[i] = ok ? bf16f(ld_stream_u16(us + c)) : 0.0f;
             }
         }
 #pragma unroll
-        for (int i = 0; i < GEMV_G; ++i) {
+        for (int i = 0; i < G; ++i) {
             if (g0 + i < nit) {
 #pragma unroll
-                for (int t = 0; t < NT; ++t) {
-                    if (t < T) {
-                        float da = chunk_dot<W, VT>(wg[i], xs + t * xstride, g0 + i, lane);
-                        float du = chunk_dot<W, VT>(wu[i], xs + t * xstride, g0 + i, lane);
-                        if constexpr (W == DT_INT4) { da *= sg[i]; du *= su[i]; }
-                        a[t] += da;
-                        u[t] += du;
-                    }
+                for (int t = 0; t < T; ++t) {
+                    a[t] = chunk_dot_s<W, VT>(wg[i], sg[i], xs + t * xstride, g0 + i, lane, a[t]);
+                    u[t] = chunk_dot_s<W, VT>(wu[i], su[i], xs + t * xstride, g0 + i, lane, u[t]);
                 }
             }
         }

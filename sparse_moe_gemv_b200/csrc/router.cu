@@ -31,18 +31,26 @@ __global__ void __launch_bounds__(RL_THREADS) router_logits_kernel(const void* x
     const int xstride = staged_bytes(H, RT, XT) / 16;
     const int t0 = blockIdx.y * RL_TOK;
     const int nt = min(RL_TOK, T - t0);
-    for (int t = 0; t < nt; ++t)
-        stage_vec<RT, XT>(xs + t * xstride, static_cast<const char*>(x) + size_t(t0 + t) * H * vbytes(XT), H, false);
+    for (int t = 0; t < RL_TOK; ++t) {
+        if (t < nt) {
+            stage_vec<RT, XT>(xs + t * xstride, static_cast<const char*>(x) + size_t(t0 + t) * H * vbytes(XT), H, false);
+        } else {
+            for (int i = threadIdx.x; i < xstride; i += blockDim.x) xs[t * xstride + i] = make_uint4(0u, 0u, 0u, 0u);
+        }
+    }
     __syncthreads();
     const int lane = threadIdx.x & 31;
     const int e = blockIdx.x * RL_WARPS + (threadIdx.x >> 5);
     if (e >= E) return;
-    float acc[RL_TOK] = {0.f, 0.f, 0.f, 0.f};
-    row_dots<RT, XT>(static_cast<const char*>(wr) + size_t(e) * row_bytes(RT, H), nullptr, H, xs, xstride, nt, lane, acc);
+    float2 acc[RL_TOK];
+#pragma unroll
+    for (int t = 0; t < RL_TOK; ++t) acc[t] = make_float2(0.f, 0.f);
+    row_dots<RT, XT, RL_TOK>(static_cast<const char*>(wr) + size_t(e) * row_bytes(RT, H), nullptr, H / Wv<RT>::V, xs,
+                             xstride, lane, acc);
     const float b = bias ? bias[e] : 0.0f;
 #pragma unroll
     for (int t = 0; t < RL_TOK; ++t) {
-        const float v = warp_sum(acc[t]);
+        const float v = warp_sum(acc[t].x + acc[t].y);
         if (lane == 0 && t < nt) logits[size_t(t0 + t) * E + e] = v + b;
     }
 }
@@ -51,10 +59,11 @@ template <int XT, int RT>
 __global__ void __launch_bounds__(RL_THREADS) topk_kernel(const float* logits, int T, int E, int k, const void* x,
                                                           const void* g, int H, int32_t* ids, float* w,
                                                           float* sgate, float* zero_out) {
+    extern __shared__ __align__(16) uint32_t keys[];  // [RL_WARPS][E]
     const int lane = threadIdx.x & 31;
     const int t = blockIdx.x * RL_WARPS + (threadIdx.x >> 5);
     if (t >= T) return;
-    warp_topk(logits + size_t(t) * E, E, k, ids + size_t(t) * k, w + size_t(t) * k);
+    warp_topk(logits + size_t(t) * E, E, k, keys + (threadIdx.x >> 5) * E, ids + size_t(t) * k, w + size_t(t) * k);
     float acc = 0.0f;
     for (int h = lane; h < H; h += 32) {
         float xv, gv;
@@ -88,7 +97,11 @@ redmoe_status launch_router_dt(const redmoe_layer* L, const void* x, int T, floa
         if (cudaGetLastError() != cudaSuccess) return REDMOE_ERR_CUDA;
         if (launches) *launches += 1;
     }
-    topk_kernel<XT, RT><<<(T + RL_WARPS - 1) / RL_WARPS, RL_THREADS, 0, stream>>>(
+    const int ksmem = RL_WARPS * E * 4;
+    if (ksmem > 48 * 1024 &&
+        cudaFuncSetAttribute(topk_kernel<XT, RT>, cudaFuncAttributeMaxDynamicSharedMemorySize, ksmem) != cudaSuccess)
+        return REDMOE_ERR_CUDA;
+    topk_kernel<XT, RT><<<(T + RL_WARPS - 1) / RL_WARPS, RL_THREADS, ksmem, stream>>>(
         logits, T, E, L->top_k, x, L->shared_gate_w, H, ids, w, sgate, zero_out);
     if (cudaGetLastError() != cudaSuccess) return REDMOE_ERR_CUDA;
     if (launches) *launches += 1;
