@@ -157,6 +157,24 @@ redmoe_status redmoe_forward_stack(const redmoe_layer *layers, int32_t n_layers,
                                    int32_t *const *ids, float *const *ws, void *workspace,
                                    size_t workspace_bytes, void *stream);
 
+/* redmoe_forward for decode sizes (1 <= T <= 4) without a caller workspace, for callers
+ * that cannot allocate device memory: code inside a strict CUDA stream capture (where an
+ * allocation breaks the capture), latency-critical loops that must not touch the
+ * allocator, or plug-ins whose host framework owns the whole device memory budget.
+ * There is no counterpart on the pages; it is a deployment convenience of this library.
+ *
+ * The scratch memory is a fixed 1 MiB array inside the library image; every GPU that
+ * loads the library holds it until the process exits. Arguments and outputs are those of
+ * redmoe_forward. The first call on each device looks up the array's device address
+ * (cudaGetSymbolAddress, with that device current): make that first call outside any
+ * stream capture. Each call clears the array's control block with an async memset
+ * before the kernel; nothing is allocated or freed. All calls on a device share the
+ * array, so calls that can overlap on the GPU race and must not be made; order them on
+ * one stream. Returns REDMOE_ERR_WORKSPACE if the layer at this T needs more than the
+ * 1 MiB scratch, REDMOE_ERR_UNSUPPORTED for T > 4, otherwise as redmoe_forward. */
+redmoe_status redmoe_forward_noalloc(const redmoe_layer *L, const void *x, int32_t T, float *out,
+                                     int32_t *topk_ids, float *topk_w, void *stream);
+
 /* Synchronise `stream`, then read the workspace's error word: REDMOE_ERR_TIMEOUT if an
  * in-kernel grid barrier gave up waiting (bounded at about one second) since the last
  * redmoe_workspace_init, else REDMOE_OK. REDMOE_ERR_CUDA if the stream reports an error. */

@@ -27,7 +27,7 @@ STATUS = {0: "REDMOE_OK", 1: "REDMOE_ERR_INVALID_ARG", 2: "REDMOE_ERR_UNSUPPORTE
 # entry points declared in include/redmoe.h
 SYMBOLS = ("redmoe_abi_version", "redmoe_status_string", "redmoe_workspace_bytes", "redmoe_workspace_init",
            "redmoe_forward", "redmoe_router", "redmoe_route_build", "redmoe_forward_stack",
-           "redmoe_check_timeout")
+           "redmoe_check_timeout", "redmoe_forward_noalloc")
 
 _lock = threading.Lock()
 _lib = None
@@ -84,6 +84,8 @@ def load():
         lib.redmoe_forward_stack.argtypes = [P, i32, P, i32, P, P, P, P, sz, P]
         lib.redmoe_check_timeout.restype = i32
         lib.redmoe_check_timeout.argtypes = [P, P]
+        lib.redmoe_forward_noalloc.restype = i32
+        lib.redmoe_forward_noalloc.argtypes = [P, P, i32, P, P, P, P]
         if lib.redmoe_abi_version() != ABI_VERSION:
             raise RuntimeError("libredmoe.so ABI version mismatch")
         _lib = lib
@@ -214,3 +216,18 @@ def redmoe_forward_stack(layers: Sequence[Layer], xs: Sequence[torch.Tensor], ou
 
 def redmoe_check_timeout(workspace: torch.Tensor, stream=None) -> None:
     _check(load().redmoe_check_timeout(_ptr(workspace), _stream(stream)), "redmoe_check_timeout")
+
+
+def redmoe_forward_noalloc(layer: Layer, x: torch.Tensor, out: torch.Tensor, topk_ids: torch.Tensor,
+                           topk_w: torch.Tensor, stream=None) -> None:
+    """redmoe_forward for 1..4 token rows without a workspace argument.
+
+    For callers that cannot allocate device memory (a strict stream capture, a loop that
+    must not touch the allocator, a plug-in without a memory budget of its own): the
+    scratch is a fixed 1 MiB array inside the library, shared by every call on the
+    device. Calls must not overlap on the GPU; the first call on a device must not be
+    made inside a stream capture (it looks up the array's address).
+    """
+    st = load().redmoe_forward_noalloc(layer.ref, _ptr(x), int(x.shape[0]), _ptr(out), _ptr(topk_ids),
+                                       _ptr(topk_w), _stream(stream))
+    _check(st, "redmoe_forward_noalloc")

@@ -131,6 +131,10 @@ redmoe_status check_ws(const redmoe_layer* L, int T, const void* ws, size_t byte
 redmoe_status cuda_ok(cudaError_t e) { return e == cudaSuccess ? REDMOE_OK : REDMOE_ERR_CUDA; }
 
 }  // namespace
+
+// Layer validation for redmoe_forward_noalloc (same rules as the other entry points).
+redmoe_status check_layer_for_noalloc(const redmoe_layer* L) { return check_layer(L); }
+
 }  // namespace redmoe
 
 using namespace redmoe;

@@ -135,3 +135,15 @@ def test_router_and_stack_reject_bad_arguments(lib):
     assert lib.redmoe_forward_stack(None, 2, None, 1, None, None, None, FAKE, 1 << 30, 0) == INVALID
     assert lib.redmoe_workspace_init(None, 256, 0) == WORKSPACE
     assert lib.redmoe_check_timeout(None, 0) == WORKSPACE
+
+
+def test_noalloc_rejects_before_touching_cuda(lib):
+    L = _layer()
+    f = lib.redmoe_forward_noalloc
+    assert f(C.byref(L), FAKE, -1, FAKE, FAKE, FAKE, 0) == INVALID
+    assert f(C.byref(L), None, 1, FAKE, FAKE, FAKE, 0) == INVALID
+    assert f(C.byref(L), FAKE, 5, FAKE, FAKE, FAKE, 0) == UNSUPPORTED
+    assert f(C.byref(L), FAKE, 0, FAKE, FAKE, FAKE, 0) == OK
+    # a layer whose decode scratch exceeds the fixed 1 MiB array is refused
+    big = _layer(top_k=32, inter=2048, n_experts=64)
+    assert f(C.byref(big), FAKE, 4, FAKE, FAKE, FAKE, 0) == WORKSPACE
