@@ -123,8 +123,12 @@ redmoe_status redmoe_workspace_init(void *workspace, size_t workspace_bytes, voi
  *   topk_w   [T, k] fp32, renormalised weights in the same order (sum to 1 per row)
  *   dbg      NULL, or device arrays that receive the token->expert grouping
  * T == 0 is a valid empty call: nothing is enqueued. Decode sizes (T <= 4) run one
- * persistent kernel; larger T runs the batched (grouped-GEMM) path, which needs bf16
- * x, router and experts (other dtypes at T > 4 return REDMOE_ERR_UNSUPPORTED). */
+ * persistent kernel; larger T runs the batched path: a tensor-core router GEMM, top-k,
+ * the grouping, and tensor-core grouped GEMMs for the experts (gate/up with SwiGLU,
+ * then down with a weighted fp32 scatter-add into out, whose summation order is not
+ * fixed). The batched path needs bf16 x, router and experts, shared_inter == inter,
+ * hidden % 256 == 0 and inter % 128 == 0; other layers at T > 4 return
+ * REDMOE_ERR_UNSUPPORTED. */
 redmoe_status redmoe_forward(const redmoe_layer *L, const void *x, int32_t T, float *out,
                              int32_t *topk_ids, float *topk_w, void *workspace,
                              size_t workspace_bytes, const redmoe_route_debug *dbg, void *stream);

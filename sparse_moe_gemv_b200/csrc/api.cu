@@ -116,6 +116,9 @@ size_t ws_bytes(const redmoe_layer* L, int T) {
     if (T <= DECODE_MAX_T) {
         const DecodeWs d = decode_ws_layout(T, L->n_experts, L->top_k, L->inter, L->shared_inter);
         need = d.total > need ? d.total : need;
+    } else if (batch_shape_ok(L)) {
+        const BatchLayout g = batch_layout(T, L->n_experts, L->top_k, L->hidden, L->inter);
+        need = g.total > need ? g.total : need;
     }
     const BatchWs b = batch_ws_layout(T, L->n_experts);
     need = b.total > need ? b.total : need;
@@ -178,7 +181,11 @@ redmoe_status redmoe_forward(const redmoe_layer* L, const void* x, int32_t T, fl
     if (dbg && (!dbg->counts || !dbg->offsets || !dbg->perm)) return REDMOE_ERR_INVALID_ARG;
     if ((st = check_ws(L, T, workspace, workspace_bytes)) != REDMOE_OK) return st;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    if (T > DECODE_MAX_T) return REDMOE_ERR_UNSUPPORTED;
+    if (T > DECODE_MAX_T) {
+        if (!batch_shape_ok(L)) return REDMOE_ERR_UNSUPPORTED;
+        if ((long long)T * L->top_k + T > (1ll << 30)) return REDMOE_ERR_INVALID_ARG;
+        return launch_batched(L, x, T, out, topk_ids, topk_w, workspace, dbg, s, nullptr);
+    }
     const DecLayer d = dec_layer(L, x, out, topk_ids, topk_w);
     st = launch_decode(L, &d, 1, T, workspace, s, nullptr);
     if (st != REDMOE_OK) return st;

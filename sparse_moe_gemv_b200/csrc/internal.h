@@ -50,6 +50,15 @@ DecodeWs decode_ws_layout(int T, int E, int k, int I, int Is);
 redmoe_status launch_decode(const redmoe_layer* shape, const DecLayer* layers, int n_layers, int T,
                             void* workspace, cudaStream_t stream, int* launches);
 
+// Workspace carve-up of the batched (grouped-GEMM) path (byte offsets from the base).
+struct BatchLayout {
+    size_t logits, sgate, counts, offsets, perm, tiles, xg, h, total;
+};
+BatchLayout batch_layout(int T, int E, int k, int H, int I);
+bool batch_shape_ok(const redmoe_layer* L);
+redmoe_status launch_batched(const redmoe_layer* L, const void* x, int T, float* out, int32_t* ids, float* w,
+                             void* ws, const redmoe_route_debug* dbg, cudaStream_t s, int* launches);
+
 // Device attributes cached per device.
 struct DevInfo {
     int sm_count;

@@ -52,7 +52,7 @@ def check_order(logits_row, ids):
     return bool(np.all(np.diff(l) <= GAP))
 
 
-def reference(shape, L, x_dev, gpu_ids=None):
+def reference(shape, L, x_dev, gpu_ids=None, rows=None):
     """Oracle routing + outputs for the device layer L and input x_dev.
 
     With gpu_ids given, exempt tokens take the oracle-enumerated set equal to the GPU's
@@ -79,17 +79,20 @@ def reference(shape, L, x_dev, gpu_ids=None):
         chosen = sorted(g, key=lambda e: (-r["logits"][t][e], e))
         ids[t] = chosen
         w[t] = oracle.renorm(r["logits"][t], np.array(chosen, np.int32))
-    used = sorted(set(ids.reshape(-1).tolist()))
+    rows = np.arange(T) if rows is None else np.asarray(rows)
+    used = sorted(set(ids[rows].reshape(-1).tolist()))
     lay_e = mi.layer_to_numpy(L, experts=used)
-    out = oracle.experts(lay_e, shape, x, ids, w, r["s"])
-    return dict(ids=ids, w=w, s=r["s"], out=out, logits=r["logits"], exempt=exempt, bad=bad)
+    out = oracle.experts(lay_e, shape, x[rows], ids[rows], w[rows], r["s"][rows])
+    return dict(ids=ids, w=w, s=r["s"], out=out, logits=r["logits"], exempt=exempt, bad=bad, rows=rows)
 
 
-def assert_layer_parity(shape, L, x_dev, out_gpu, ids_gpu, w_gpu, out_tol, w_tol, label=""):
+def assert_layer_parity(shape, L, x_dev, out_gpu, ids_gpu, w_gpu, out_tol, w_tol, label="", rows=None):
+    """rows: token rows whose outputs are checked (all by default); ids and weights are
+    always checked for every token."""
     ids_g = ids_gpu.detach().cpu().numpy()
     w_g = w_gpu.detach().cpu().numpy().astype(np.float64)
-    out_g = out_gpu.detach().cpu().numpy().astype(np.float64)
-    ref = reference(shape, L, x_dev, gpu_ids=ids_g)
+    ref = reference(shape, L, x_dev, gpu_ids=ids_g, rows=rows)
+    out_g = out_gpu.detach().cpu().numpy().astype(np.float64)[ref["rows"]]
     assert not ref["bad"], f"{label}: GPU top-k outside the valid near-tie sets for tokens {ref['bad']}"
     T = ids_g.shape[0]
     for t in range(T):
@@ -102,7 +105,7 @@ def assert_layer_parity(shape, L, x_dev, out_gpu, ids_gpu, w_gpu, out_tol, w_tol
     rms = float(np.sqrt(np.mean(ref["out"] ** 2)))
     err = float(np.max(np.abs(out_g - ref["out"]))) if out_g.size else 0.0
     assert err <= out_tol * rms, f"{label}: max|out err| {err:.3e} > {out_tol} * RMS {rms:.3e}"
-    return dict(err=err, rms=rms, exempt=int(ref["exempt"].sum()))
+    return dict(err=err, rms=rms, exempt=int(ref["exempt"].sum()), ref=ref)
 
 
 def tolerances(shape):
