@@ -44,6 +44,7 @@ FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
 QWEN = mi.LayerShape(H=2048, E=512, k=10, I=512, Is=512)
 QWEN_INT4 = mi.LayerShape(H=2048, E=512, k=10, I=512, Is=512, expert_dtype="int4g32")
+QWEN_ZIPF = mi.LayerShape(H=2048, E=512, k=10, I=512, Is=512, zipf_s=1.1)
 
 WORKLOADS = {
     "decode_t1": dict(shape=QWEN, T=1, layers=12, stack=False, seed=1000, kernel="decode_kernel",
@@ -54,7 +55,15 @@ WORKLOADS = {
                       desc="12 distinct Qwen3-Next-shaped bf16 layers back to back, T=3"),
     "int4_48": dict(shape=QWEN_INT4, T=1, layers=48, stack=True, seed=4000, kernel="decode_kernel",
                     desc="48 distinct Qwen3-Next-shaped layers, int4 group-32 experts, decode T=1"),
+    "prefill": dict(shape=QWEN_ZIPF, T=2048, layers=1, stack=False, seed=3000, kernel="layer (6 kernels)",
+                    desc="Qwen3-Next-shaped MoE layer, bf16, 2048-token prefill chunk, Zipf(1.1) router offsets"),
 }
+
+
+def layer_flops(shape, T):
+    """Algorithmic FLOPs of one layer call: router 2*T*E*H, routed experts 2*T*k*3*H*I,
+    shared expert 2*T*3*H*Is (multiply-adds counted as two)."""
+    return 2.0 * T * (shape.E * shape.H + shape.k * 3 * shape.H * shape.I + 3 * shape.H * shape.Is)
 
 
 # ------------------------------------------------------------------ helpers
@@ -317,6 +326,8 @@ def gpu_arm(args, wl, world, rank, local):
     B = build_workload(wl, smg)
     stream = torch.cuda.Stream()
     step, launches_per_step = make_step(wl, smg, B, stream)
+    with torch.cuda.stream(stream):
+        step(0)  # one eager call: per-device set-up (attributes, driver entry points) outside capture
     torch.cuda.synchronize()
     # graphs: one rotation of the layers per replay (stack workloads: one stack per replay)
     chunk = 1 if wl["stack"] else wl["layers"]
@@ -366,6 +377,18 @@ def gpu_arm(args, wl, world, rank, local):
     launch_s = el_ms / 1e3 / launches
     hbm, bf16, bf16_sus, src = peaks()
     achieved = bytes_per_launch / launch_s / 1e9
+    if T > 4:
+        # batched path: six kernels per step; the roofline is the tensor-core one of the layer
+        flops = layer_flops(shape, T)
+        step_s = el_ms / 1e3 / K
+        tfl = flops / step_s / 1e12
+        roof = {"bound": "tensor", "achieved": tfl, "peak": bf16, "unit": "TFLOP/s", "frac": tfl / bf16,
+                "traffic": profile_traffic(args.workload), "kernel": wl["kernel"], "flops_per_step": flops,
+                "weight_bytes_per_step": bytes_per_launch, "hbm_gbs_of_weights": bytes_per_launch / step_s / 1e9,
+                "peak_source": f"{src} (MEASURED_PEAKS.json bf16_tflops, burst)"}
+        launches = K * 6
+    else:
+        roof = None
 
     # end to end through the C ABI with pinned host buffers: per step H2D x, forward, D2H out/ids/w
     e2e = e2e_arm(args, wl, smg, B, stream, world)
@@ -379,10 +402,10 @@ def gpu_arm(args, wl, world, rank, local):
                          f"({wl['layers']} distinct layers)" if not wl["stack"] else
                          f"inputs larger than L2: {wl['layers']} distinct layers per step",
                    "parallelism": "replicas" if world > 1 else "single GPU", "timing": "CUDA graph replay"},
-        "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
-                     "traffic": profile_traffic(args.workload), "kernel": wl["kernel"],
-                     "bytes_per_launch": bytes_per_launch, "launch_us": launch_s * 1e6,
-                     "peak_source": f"{src} (MEASURED_PEAKS.json hbm_gbs)" if src == "measured" else "fallback"},
+        "roofline": roof or {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
+                             "traffic": profile_traffic(args.workload), "kernel": wl["kernel"],
+                             "bytes_per_launch": bytes_per_launch, "launch_us": launch_s * 1e6,
+                             "peak_source": f"{src} (MEASURED_PEAKS.json hbm_gbs)" if src == "measured" else "fallback"},
         "e2e": e2e,
         "gpu_launches": launches,
         "clocks": clk.summary(),
@@ -450,6 +473,7 @@ def main():
     ap.add_argument("--workload", default="decode_t1", choices=sorted(WORKLOADS))
     ap.add_argument("--impl", default="redmoe", choices=["redmoe", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-prefill", action="store_true", help="skip the prefill summary of the default run")
     ap.add_argument("--layers", type=int, default=None,
                     help="override the number of distinct layers (small cases for profiler captures)")
     args = ap.parse_args()
@@ -467,6 +491,13 @@ def main():
             torch.distributed.destroy_process_group()
         return
     res = gpu_arm(args, wl, world, rank, local)
+    if args.workload == "decode_t1" and not args.no_prefill:
+        torch.cuda.empty_cache()
+        pargs = argparse.Namespace(**{**vars(args), "steps": min(args.steps, 30), "warmup": 3, "workload": "prefill"})
+        pre = gpu_arm(pargs, WORKLOADS["prefill"], world, rank, local)
+        res["prefill"] = {"workload": WORKLOADS["prefill"]["desc"], "value": pre["value"], "unit": "tokens/s",
+                          "ms_per_step": pre["ms_per_step"], "steps": pre["steps"], "roofline": pre["roofline"],
+                          "e2e": pre["e2e"], "gpu_launches": pre["gpu_launches"], "clocks": pre["clocks"]}
     if rank == 0:
         if world == 1 and not args.no_cpu_baseline:
             res["cpu_baseline"] = cpu_oracle_sample(wl)

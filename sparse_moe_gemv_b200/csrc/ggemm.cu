@@ -40,14 +40,19 @@ constexpr int BM = 128;
 constexpr int BK = 64;
 constexpr int GEMM_THREADS = 192;
 
+constexpr int RED_COLS = 64;                    // scatter epilogue: columns per bulk reduction
+constexpr int RED_STRIDE = RED_COLS * 4 + 16;   // padded staging row (bytes): 4-way bank conflicts at most
+constexpr int RED_WARP = 2 * 32 * RED_STRIDE;   // two staging buffers of 32 rows per epilogue warp
+
 template <int MODE, int BN>
 struct Cfg {
     static constexpr int A_BYTES = BM * BK * 2;
     static constexpr int B_BYTES = BN * BK * 2;
     static constexpr int STAGE = A_BYTES + B_BYTES;
-    static constexpr int NS = (STAGE <= 24 * 1024) ? 8 : 4;
+    static constexpr int NS = (STAGE <= 24 * 1024) ? 8 : (MODE == GM_SCATTER ? 3 : 4);
     static constexpr int TMEM_COLS = (2 * BN <= 32) ? 32 : (2 * BN <= 64 ? 64 : (2 * BN <= 128 ? 128 : (2 * BN <= 256 ? 256 : 512)));
-    static constexpr int SMEM = 1024 + NS * STAGE + 256;  // alignment slack + stages + barriers
+    static constexpr int STAGING = (MODE == GM_SCATTER) ? 4 * RED_WARP : 0;
+    static constexpr int SMEM = 1024 + NS * STAGE + STAGING + 256;  // alignment slack + stages + staging + barriers
 };
 
 struct Tile {
@@ -99,18 +104,14 @@ __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" :: "r"(smem_u32(bar)) : "memory");
 }
 
-__device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float c, float d) {
-    asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" :: "l"(addr), "f"(a), "f"(b), "f"(c), "f"(d)
-                 : "memory");
-}
-
 template <int MODE, int BN>
 __global__ void __launch_bounds__(GEMM_THREADS, 1) ggemm_kernel(const __grid_constant__ GemmParams p) {
     using C = Cfg<MODE, BN>;
     constexpr int NS = C::NS;
     extern __shared__ unsigned char smem_raw[];
     unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint64_t* full = reinterpret_cast<uint64_t*>(smem + NS * C::STAGE);
+    unsigned char* staging = smem + NS * C::STAGE;
+    uint64_t* full = reinterpret_cast<uint64_t*>(staging + C::STAGING);
     uint64_t* empty = full + NS;
     uint64_t* tfull = empty + NS;
     uint64_t* tempty = tfull + 2;
@@ -137,8 +138,8 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) ggemm_kernel(const __grid_con
     const uint32_t tmem_base = *tmem_slot;
     const int total = total_tiles<MODE>(p);
 
-    if (warp == 0 && lane == 0) {
-        // ------------------------------------------------------------ producer
+    if (warp == 0) {
+        // ------------------------------------------------------------ producer (lane 0)
         uint32_t it = 0;
         for (int w = blockIdx.x; w < total; w += gridDim.x) {
             const Tile t = tile_of<MODE>(p, w);
@@ -146,8 +147,9 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) ggemm_kernel(const __grid_con
             const bool shared = (MODE != GM_ROUTER) && t.g == p.E;
             for (int kb = 0; kb < p.num_kb; ++kb, ++it) {
                 const int s = int(it % NS);
-                mbar_wait(empty + s, ((it / NS) & 1u) ^ 1u, err, to);
                 unsigned char* st = smem + s * C::STAGE;
+                if (lane != 0) continue;
+                mbar_wait(empty + s, ((it / NS) & 1u) ^ 1u, err, to);
                 mbar_arrive_expect_tx(full + s, C::STAGE);
                 tma_load_2d(st, &p.tmA, kb * BK, rowA, full + s);
                 unsigned char* sb = st + C::A_BYTES;
@@ -166,8 +168,9 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) ggemm_kernel(const __grid_con
         }
         // drain: wait until every stage issued here has landed (consumed or not)
         const uint32_t n_issued = it;
-        for (uint32_t j = (n_issued > uint32_t(NS) ? n_issued - NS : 0u); j < n_issued; ++j)
-            mbar_wait(full + (j % NS), (j / NS) & 1u, err, to);
+        if (lane == 0)
+            for (uint32_t j = (n_issued > uint32_t(NS) ? n_issued - NS : 0u); j < n_issued; ++j)
+                mbar_wait(full + (j % NS), (j / NS) & 1u, err, to);
     } else if (warp == 1 && lane == 0) {
         // ------------------------------------------------------------ MMA issuer
         constexpr uint32_t idesc = idesc_bf16_f32(BM, BN);
@@ -196,6 +199,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) ggemm_kernel(const __grid_con
         const int q = warp & 3;              // TMEM lane quadrant of this warp
         const int r = q * 32 + lane;         // row within the tile
         uint32_t tc = 0;
+        uint32_t red_chunk = 0;              // scatter: staging buffer sequence
         for (int w = blockIdx.x; w < total; w += gridDim.x, ++tc) {
             const Tile t = tile_of<MODE>(p, w);
             const uint32_t acc = tc & 1u;
@@ -238,6 +242,8 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) ggemm_kernel(const __grid_con
                     }
                 }
             } else {
+                // weight * y for this row, staged in shared memory (a padded row per thread,
+                // two buffers per warp) and added into out[token] by 256-byte bulk reductions
                 int tok = 0;
                 float wgt = 0.0f;
                 if (valid) {
@@ -250,22 +256,29 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) ggemm_kernel(const __grid_con
                         wgt = __ldg(p.sgate + lr);
                     }
                 }
+                unsigned char* wbuf = staging + (warp - 2) * RED_WARP;
 #pragma unroll 1
-                for (int c = 0; c < BN / 32; ++c) {
-                    float v[32];
-                    tmem_ld32(taddr + c * 32, v);
-                    if (valid) {
-                        float* dst = p.out_f32 + size_t(tok) * p.N + t.n * BN + c * 32;
+                for (int c = 0; c < BN / RED_COLS; ++c, ++red_chunk) {
+                    float v[32], u[32];
+                    tmem_ld32(taddr + c * RED_COLS, v);
+                    tmem_ld32(taddr + c * RED_COLS + 32, u);
+                    unsigned char* row = wbuf + (red_chunk & 1u) * (32 * RED_STRIDE) + lane * RED_STRIDE;
+                    bulk_wait_read<1>();  // the buffer used two chunks ago has been read
+                    float4* r4 = reinterpret_cast<float4*>(row);
 #pragma unroll
-                        for (int j = 0; j < 8; ++j)
-                            red_add_v4(dst + 4 * j, wgt * v[4 * j], wgt * v[4 * j + 1], wgt * v[4 * j + 2], wgt * v[4 * j + 3]);
-                    }
+                    for (int j = 0; j < 8; ++j) r4[j] = make_float4(wgt * v[4 * j], wgt * v[4 * j + 1], wgt * v[4 * j + 2], wgt * v[4 * j + 3]);
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) r4[8 + j] = make_float4(wgt * u[4 * j], wgt * u[4 * j + 1], wgt * u[4 * j + 2], wgt * u[4 * j + 3]);
+                    fence_proxy_async_smem();
+                    if (valid) bulk_reduce_add_f32(p.out_f32 + size_t(tok) * p.N + t.n * BN + c * RED_COLS, row, RED_COLS * 4);
+                    bulk_commit();
                 }
             }
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(tempty + acc);
         }
+        if (MODE == GM_SCATTER) bulk_wait<0>();  // every bulk reduction of this thread has completed
     }
     tc_fence_before();
     __syncthreads();
