@@ -55,7 +55,7 @@ WORKLOADS = {
                       desc="12 distinct Qwen3-Next-shaped bf16 layers back to back, T=3"),
     "int4_48": dict(shape=QWEN_INT4, T=1, layers=48, stack=True, seed=4000, kernel="decode_kernel",
                     desc="48 distinct Qwen3-Next-shaped layers, int4 group-32 experts, decode T=1"),
-    "prefill": dict(shape=QWEN_ZIPF, T=2048, layers=1, stack=False, seed=3000, kernel="layer (6 kernels)",
+    "prefill": dict(shape=QWEN_ZIPF, T=2048, layers=1, stack=False, seed=3000, kernel="layer (4 kernels)",
                     desc="Qwen3-Next-shaped MoE layer, bf16, 2048-token prefill chunk, Zipf(1.1) router offsets"),
 }
 
@@ -378,7 +378,7 @@ def gpu_arm(args, wl, world, rank, local):
     hbm, bf16, bf16_sus, src = peaks()
     achieved = bytes_per_launch / launch_s / 1e9
     if T > 4:
-        # batched path: six kernels per step; the roofline is the tensor-core one of the layer
+        # batched path: four kernels per step; the roofline is the tensor-core one of the layer
         flops = layer_flops(shape, T)
         step_s = el_ms / 1e3 / K
         tfl = flops / step_s / 1e12
@@ -386,7 +386,7 @@ def gpu_arm(args, wl, world, rank, local):
                 "traffic": profile_traffic(args.workload), "kernel": wl["kernel"], "flops_per_step": flops,
                 "weight_bytes_per_step": bytes_per_launch, "hbm_gbs_of_weights": bytes_per_launch / step_s / 1e9,
                 "peak_source": f"{src} (MEASURED_PEAKS.json bf16_tflops, burst)"}
-        launches = K * 6
+        launches = K * 4
     else:
         roof = None
 

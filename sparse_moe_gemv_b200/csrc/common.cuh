@@ -123,15 +123,18 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
     return ok != 0;
 }
 // Bounded wait for the phase of `bar` with the given parity. Gives up after timeout_ns
-// (or at once if another thread has already recorded a timeout): sets ERRBIT_TIMEOUT in
-// *err and returns false; the caller carries on with whatever the buffer holds.
+// (or, once it has waited 20 us, as soon as another thread has recorded a timeout): sets
+// ERRBIT_TIMEOUT in *err and returns false; the caller carries on with whatever the buffer
+// holds. The error word is not read during the first 20 us: a global load in the polling
+// loop would delay noticing a completed phase by its latency.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* err, uint64_t timeout_ns) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer_ns();
     for (uint32_t i = 1;; ++i) {
         if (mbar_try_wait(bar, parity)) return true;
         if ((i & 63u) == 0u) {
-            if (ld_relaxed_gpu(err) != 0 || globaltimer_ns() - t0 > timeout_ns || i > (1u << 26)) {
+            const uint64_t dt = globaltimer_ns() - t0;
+            if (dt > timeout_ns || i > (1u << 26) || (dt > 20000u && ld_relaxed_gpu(err) != 0)) {
                 atomicOr(err, ERRBIT_TIMEOUT);
                 return false;
             }
@@ -170,7 +173,8 @@ __device__ __forceinline__ void grid_barrier(Control* ctl, unsigned nblocks, uns
             const uint64_t t0 = globaltimer_ns();
             for (uint32_t spins = 1; ld_acquire_gpu(&ctl->bar_count) < target; ++spins) {
                 if ((spins & 63u) == 0u) {
-                    if (ld_relaxed_gpu(&ctl->err) != 0 || globaltimer_ns() - t0 > timeout_ns || spins > (1u << 26)) {
+                    const uint64_t dt = globaltimer_ns() - t0;
+                    if (dt > timeout_ns || spins > (1u << 26) || (dt > 20000u && ld_relaxed_gpu(&ctl->err) != 0)) {
                         atomicOr(&ctl->err, ERRBIT_TIMEOUT);
                         break;
                     }
@@ -198,7 +202,8 @@ __device__ __forceinline__ void grid_wait(Control* ctl, unsigned nblocks, unsign
             const uint64_t t0 = globaltimer_ns();
             for (uint32_t spins = 1; ld_acquire_gpu(&ctl->bar_count) < target; ++spins) {
                 if ((spins & 63u) == 0u) {
-                    if (ld_relaxed_gpu(&ctl->err) != 0 || globaltimer_ns() - t0 > timeout_ns || spins > (1u << 26)) {
+                    const uint64_t dt = globaltimer_ns() - t0;
+                    if (dt > timeout_ns || spins > (1u << 26) || (dt > 20000u && ld_relaxed_gpu(&ctl->err) != 0)) {
                         atomicOr(&ctl->err, ERRBIT_TIMEOUT);
                         break;
                     }

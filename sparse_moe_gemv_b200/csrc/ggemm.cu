@@ -51,7 +51,9 @@ struct Cfg {
     static constexpr int STAGE = A_BYTES + B_BYTES;
     static constexpr int NS = (STAGE <= 24 * 1024) ? 8 : (MODE == GM_SCATTER ? 3 : 4);
     static constexpr int TMEM_COLS = (2 * BN <= 32) ? 32 : (2 * BN <= 64 ? 64 : (2 * BN <= 128 ? 128 : (2 * BN <= 256 ? 256 : 512)));
-    static constexpr int STAGING = (MODE == GM_SCATTER) ? 4 * RED_WARP : 0;
+    // scatter: weighted rows for the bulk reductions; router: a 32 x 33 fp32 transpose
+    // buffer per epilogue warp
+    static constexpr int STAGING = (MODE == GM_SCATTER) ? 4 * RED_WARP : (MODE == GM_ROUTER ? 4 * 32 * 33 * 4 : 0);
     static constexpr int SMEM = 1024 + NS * STAGE + STAGING + 256;  // alignment slack + stages + staging + barriers
 };
 
@@ -151,7 +153,8 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) ggemm_kernel(const __grid_con
                 if (lane != 0) continue;
                 mbar_wait(empty + s, ((it / NS) & 1u) ^ 1u, err, to);
                 mbar_arrive_expect_tx(full + s, C::STAGE);
-                tma_load_2d(st, &p.tmA, kb * BK, rowA, full + s);
+                if (MODE == GM_SWIGLU && shared) tma_load_2d(st, &p.tmA2, kb * BK, t.m * BM, full + s);
+                else tma_load_2d(st, &p.tmA, kb * BK, rowA, full + s);
                 unsigned char* sb = st + C::A_BYTES;
                 if (MODE == GM_SWIGLU) {
                     const int nh = t.n * (BN / 2);
@@ -210,17 +213,26 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) ggemm_kernel(const __grid_con
             const bool valid = lr < t.C;
             const int grow = t.S + lr;       // row in the grouped row space
             if (MODE == GM_ROUTER) {
+                // this warp's 32 rows x 32 columns go through a padded shared buffer, so
+                // that each store instruction writes one row's 128 contiguous bytes
+                float* tb = reinterpret_cast<float*>(staging) + (warp - 2) * (32 * 33);
+                const int row0 = t.m * BM + q * 32;
 #pragma unroll 1
                 for (int c = 0; c < BN / 32; ++c) {
                     float v[32];
                     tmem_ld32(taddr + c * 32, v);
                     const int n0 = t.n * BN + c * 32;
-                    if (valid) {
-                        float* dst = p.out_f32 + size_t(grow) * p.N + n0;
 #pragma unroll
-                        for (int j = 0; j < 32; ++j)
-                            if (n0 + j < p.N) dst[j] = v[j] + (p.bias ? __ldg(p.bias + n0 + j) : 0.0f);
+                    for (int j = 0; j < 32; ++j) tb[lane * 33 + j] = v[j];
+                    __syncwarp();
+                    const int n = n0 + lane;
+                    const float b = (p.bias && n < p.N) ? __ldg(p.bias + n) : 0.0f;
+#pragma unroll 4
+                    for (int i = 0; i < 32; ++i) {
+                        const int row = row0 + i;
+                        if (row < t.C && n < p.N) p.out_f32[size_t(row) * p.N + n] = tb[i * 33 + lane] + b;
                     }
+                    __syncwarp();
                 }
             } else if (MODE == GM_SWIGLU) {
 #pragma unroll 1

@@ -12,6 +12,7 @@ enum : int { GM_ROUTER = 0, GM_SWIGLU = 1, GM_SCATTER = 2 };
 
 struct GemmParams {
     CUtensorMap tmA;    // A rows [rows, K]
+    CUtensorMap tmA2;   // SWIGLU: the shared expert's A rows (x itself, [T, K])
     CUtensorMap tmB0;   // routed B rows (SWIGLU: gate), or the router weights
     CUtensorMap tmB1;   // routed up rows (SWIGLU only)
     CUtensorMap tmS0;   // shared-expert B rows (SWIGLU: gate)

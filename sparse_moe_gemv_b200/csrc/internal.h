@@ -14,6 +14,7 @@ constexpr int MAX_TOPK = 32;
 constexpr int MAX_EXPERTS = 1024;
 constexpr int MAX_STACK = 64;          // layers per persistent decode launch
 constexpr uint64_t BARRIER_TIMEOUT_NS = 1000000000ull;  // 1 s
+constexpr int ROUTE_MAX_BLOCKS = 256;  // blocks of the batched routing kernel, at most
 
 inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
@@ -52,7 +53,7 @@ redmoe_status launch_decode(const redmoe_layer* shape, const DecLayer* layers, i
 
 // Workspace carve-up of the batched (grouped-GEMM) path (byte offsets from the base).
 struct BatchLayout {
-    size_t logits, sgate, counts, offsets, perm, tiles, xg, h, total;
+    size_t logits, sgate, counts, offsets, perm, tiles, bhist, xg, h, total;
 };
 BatchLayout batch_layout(int T, int E, int k, int H, int I);
 bool batch_shape_ok(const redmoe_layer* L);

@@ -31,6 +31,7 @@ namespace {
 
 constexpr int RB_THREADS = 1024;
 constexpr int RB_WARPS = RB_THREADS / 32;
+constexpr int RB_BATCH = 8;  // batches of 32 ids loaded together per warp
 
 // Exclusive scan of v over the block (1024 threads); returns the block total in *total.
 __device__ int block_exclusive_scan(int v, int* warp_sums, int* total) {
@@ -74,9 +75,17 @@ __global__ void __launch_bounds__(RB_THREADS) route_build_kernel(const int32_t* 
 
     for (int i = threadIdx.x; i < RB_WARPS * E; i += RB_THREADS) hist[i] = 0;
     __syncthreads();
-    for (int i = lo + lane; i < hi; i += 32) {
-        const int e = ids[i];
-        if (e >= 0 && e < E) atomicAdd(&hist[warp * E + e], 1);
+    // ids are read RB_BATCH batches of 32 at a time: independent loads issued together
+    for (int base = lo; base < hi; base += 32 * RB_BATCH) {
+        int ev[RB_BATCH];
+#pragma unroll
+        for (int b = 0; b < RB_BATCH; ++b) {
+            const int i = base + 32 * b + lane;
+            ev[b] = i < hi ? __ldg(ids + i) : -1;
+        }
+#pragma unroll
+        for (int b = 0; b < RB_BATCH; ++b)
+            if (ev[b] >= 0 && ev[b] < E) atomicAdd(&hist[warp * E + ev[b]], 1);
     }
     __syncthreads();
     // per expert: exclusive prefix over warps, total count
@@ -110,18 +119,26 @@ __global__ void __launch_bounds__(RB_THREADS) route_build_kernel(const int32_t* 
     }
     // stable placement
     const unsigned lt = (1u << lane) - 1u;
-    for (int base = lo; base < hi; base += 32) {
-        const int i = base + lane;
-        const bool in = i < hi;
-        int e = in ? ids[i] : -1;
-        const bool ok = in && e >= 0 && e < E;
-        if (!ok) e = -1;
-        const unsigned peers = __match_any_sync(FULL, e);
-        const int rank = __popc(peers & lt);
-        if (ok) perm[offs[e] + hist[warp * E + e] + rank] = i;
-        __syncwarp();
-        if (ok && lane == 31 - __clz(peers)) hist[warp * E + e] += __popc(peers);
-        __syncwarp();
+    for (int base0 = lo; base0 < hi; base0 += 32 * RB_BATCH) {
+        int ev[RB_BATCH];
+#pragma unroll
+        for (int b = 0; b < RB_BATCH; ++b) {
+            const int i = base0 + 32 * b + lane;
+            ev[b] = i < hi ? __ldg(ids + i) : -1;
+        }
+#pragma unroll
+        for (int b = 0; b < RB_BATCH; ++b) {
+            const int i = base0 + 32 * b + lane;
+            int e = ev[b];
+            const bool ok = i < hi && e >= 0 && e < E;
+            if (!ok) e = -1;
+            const unsigned peers = __match_any_sync(FULL, e);
+            const int rank = __popc(peers & lt);
+            if (ok) perm[offs[e] + hist[warp * E + e] + rank] = i;
+            __syncwarp();
+            if (ok && lane == 31 - __clz(peers)) hist[warp * E + e] += __popc(peers);
+            __syncwarp();
+        }
     }
     (void)k;
 }

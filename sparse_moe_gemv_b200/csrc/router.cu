@@ -65,13 +65,39 @@ __global__ void __launch_bounds__(RL_THREADS) topk_kernel(const float* logits, i
     if (t >= T) return;
     warp_topk(logits + size_t(t) * E, E, k, keys + (threadIdx.x >> 5) * E, ids + size_t(t) * k, w + size_t(t) * k);
     float acc = 0.0f;
-    for (int h = lane; h < H; h += 32) {
-        float xv, gv;
-        if constexpr (XT == DT_BF16) xv = bf16f(static_cast<const uint16_t*>(x)[size_t(t) * H + h]);
-        else xv = static_cast<const float*>(x)[size_t(t) * H + h];
-        if constexpr (RT == DT_BF16) gv = bf16f(static_cast<const uint16_t*>(g)[h]);
-        else gv = static_cast<const float*>(g)[h];
-        acc = fmaf(xv, gv, acc);
+    if constexpr (XT == DT_BF16 && RT == DT_BF16) {
+        // 16-byte loads, eight chunks of 8 elements per lane issued together (H % 8 == 0)
+        const uint4* xr = reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(x) + size_t(t) * H);
+        const uint4* gr = reinterpret_cast<const uint4*>(g);
+        const int nc = H / 8;
+        for (int c0 = 0; c0 < nc; c0 += 32 * 8) {
+            uint4 xv[8], gv[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const int c = c0 + 32 * i + lane;
+                xv[i] = c < nc ? __ldg(xr + c) : make_uint4(0u, 0u, 0u, 0u);
+                gv[i] = c < nc ? __ldg(gr + c) : make_uint4(0u, 0u, 0u, 0u);
+            }
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const uint32_t xa[4] = {xv[i].x, xv[i].y, xv[i].z, xv[i].w};
+                const uint32_t ga[4] = {gv[i].x, gv[i].y, gv[i].z, gv[i].w};
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    acc = fmaf(bf16f(uint16_t(xa[j] & 0xffffu)), bf16f(uint16_t(ga[j] & 0xffffu)), acc);
+                    acc = fmaf(bf16f(uint16_t(xa[j] >> 16)), bf16f(uint16_t(ga[j] >> 16)), acc);
+                }
+            }
+        }
+    } else {
+        for (int h = lane; h < H; h += 32) {
+            float xv, gv;
+            if constexpr (XT == DT_BF16) xv = bf16f(static_cast<const uint16_t*>(x)[size_t(t) * H + h]);
+            else xv = static_cast<const float*>(x)[size_t(t) * H + h];
+            if constexpr (RT == DT_BF16) gv = bf16f(static_cast<const uint16_t*>(g)[h]);
+            else gv = static_cast<const float*>(g)[h];
+            acc = fmaf(xv, gv, acc);
+        }
     }
     acc = warp_sum(acc);
     if (lane == 0 && sgate) sgate[t] = 1.0f / (1.0f + expf(-acc));

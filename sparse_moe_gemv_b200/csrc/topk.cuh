@@ -17,12 +17,12 @@ namespace redmoe {
 // Writes ids[0..k) and the renormalised weights w_j = exp(l_j - l_0) / sum_j' exp(l_j' - l_0)
 // (the softmax over all experts, restricted to the selection and renormalised, equals the
 // softmax over the selected logits).
+//
+// warp_topk_core takes the keys in registers (key[i] of lane L is expert i * 32 + L, 0 past
+// E) and leaves the j-th selection in lane j (< k): its id and its weight.
 template <int EPL>
-__device__ __forceinline__ void warp_topk_reg(int E, int k, const uint32_t* keys, int* ids, float* wts) {
+__device__ __forceinline__ void warp_topk_core(uint32_t (&key)[EPL], int k, int& out_id, float& out_w) {
     const int lane = threadIdx.x & 31;
-    uint32_t key[EPL];
-#pragma unroll
-    for (int i = 0; i < EPL; ++i) key[i] = (i * 32 + lane < E) ? keys[i * 32 + lane] : 0u;
     uint32_t best = 0u;
     int bi = 0;
 #pragma unroll
@@ -49,9 +49,22 @@ __device__ __forceinline__ void warp_topk_reg(int E, int k, const uint32_t* keys
     const float l0 = __shfl_sync(FULL, mylogit, 0);
     const float ex = (lane < k) ? expf(mylogit - l0) : 0.0f;
     const float sum = warp_sum(ex);
+    out_id = myid;
+    out_w = ex / sum;
+}
+
+template <int EPL>
+__device__ __forceinline__ void warp_topk_reg(int E, int k, const uint32_t* keys, int* ids, float* wts) {
+    const int lane = threadIdx.x & 31;
+    uint32_t key[EPL];
+#pragma unroll
+    for (int i = 0; i < EPL; ++i) key[i] = (i * 32 + lane < E) ? keys[i * 32 + lane] : 0u;
+    int id;
+    float wv;
+    warp_topk_core<EPL>(key, k, id, wv);
     if (lane < k) {
-        ids[lane] = myid;
-        wts[lane] = ex / sum;
+        ids[lane] = id;
+        wts[lane] = wv;
     }
 }
 
