@@ -22,7 +22,8 @@
 // 16 bytes of activations and the weight bytes that multiply them), in short rolled
 // loops: at this size the cost is latency and instruction fetch, not arithmetic. The first
 // stages of phase C (whose weights do not depend on h) are issued before the barrier that
-// precedes it, and its rows are prefetched into L2 during phase B.
+// precedes it. (Prefetching all of phase C's rows into L2 during phase B measured slower at
+// T = 1: the prefetch competes with the gate/up stream for HBM.)
 //
 // Down rows are only 512 elements long (1 KiB in bf16, 256 B in int4): a phase-C stage
 // holds two rows of one expert, the lesson of the narrow-row kernel in "Research notes,
