@@ -201,6 +201,13 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) ggemm_kernel(const __grid_con
         // ------------------------------------------------------------ epilogue
         const int q = warp & 3;              // TMEM lane quadrant of this warp
         const int r = q * 32 + lane;         // row within the tile
+        if (MODE == GM_ROUTER && p.zero_out) {
+            // the output of the down GEMM, zeroed while the first tiles load
+            float4* z = reinterpret_cast<float4*>(p.zero_out);
+            const uint64_t nth = uint64_t(gridDim.x) * 128;
+            for (uint64_t i = uint64_t(blockIdx.x) * 128 + (threadIdx.x - 64); i < p.zero_f4; i += nth)
+                z[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+        }
         uint32_t tc = 0;
         uint32_t red_chunk = 0;              // scatter: staging buffer sequence
         for (int w = blockIdx.x; w < total; w += gridDim.x, ++tc) {

@@ -31,6 +31,8 @@ struct GemmParams {
     const int* perm;    // SCATTER: grouped row -> t*k + j
     const float* topk_w;// SCATTER: [T * k]
     const float* sgate; // SCATTER: [T]
+    float* zero_out;    // ROUTER: zeroed by the epilogue warps before their tiles (or null)
+    uint64_t zero_f4;   // ROUTER: float4 count of zero_out
     Control* ctl;
     uint64_t timeout_ns;
 };

@@ -1,8 +1,9 @@
 // Batched path (T > 4 token rows, bf16): the whole layer as four kernels on one stream.
 //
-//   1 router logits   tensor-core GEMM  x[T,H] . Wr[E,H]^T (+ b)      -> logits [T,E] fp32
+//   1 router logits   tensor-core GEMM  x[T,H] . Wr[E,H]^T (+ b)      -> logits [T,E] fp32;
+//                     its epilogue warps also zero out, which step 4 adds into
 //   2 routing         one cooperative kernel (route.cu): top-k, renormalised weights,
-//                     sigmoid(x . g), zeroed output rows; the stable counting sort of the
+//                     sigmoid(x . g); the stable counting sort of the
 //                     T*k rows by expert (counts, offsets, perm) and the GEMM tile schedule;
 //                     and xg, the x rows in grouped order (row offsets[e] + r of expert e is
 //                     token perm[offsets[e] + r] / k). Loading these rows inside the GEMM
@@ -30,7 +31,7 @@ redmoe_status gemm_router(GemmParams& p, cudaStream_t s);
 redmoe_status gemm_swiglu(GemmParams& p, cudaStream_t s);
 redmoe_status gemm_scatter(GemmParams& p, cudaStream_t s);
 redmoe_status launch_route(const redmoe_layer* L, const void* x, int T, const float* logits, int32_t* ids, float* w,
-                           float* sgate, float* out, int32_t* counts, int32_t* offsets, int32_t* perm, int tile_m,
+                           float* sgate, int32_t* counts, int32_t* offsets, int32_t* perm, int tile_m,
                            int32_t* tiles, void* xg, int32_t* bhist, Control* ctl, cudaStream_t stream,
                            int* launches);
 
@@ -80,10 +81,11 @@ redmoe_status launch_batched(const redmoe_layer* L, const void* x, int T, float*
         return REDMOE_ERR_CUDA;
     gr.E = E; gr.T = T; gr.k = k; gr.N = E; gr.Nb = E; gr.n_tiles = (E + 63) / 64; gr.num_kb = H / 64;
     gr.out_f32 = logits; gr.bias = L->router_bias; gr.ctl = ctl;
+    gr.zero_out = out; gr.zero_f4 = uint64_t(T) * H / 4;
     if ((st = gemm_router(gr, s)) != REDMOE_OK) return st;
     if (launches) *launches += 1;
     // 2 routing: top-k, weights, shared gate, zeroed out, grouping, tile schedule, gathered x
-    if ((st = launch_route(L, x, T, logits, ids, w, sgate, out, counts, offsets, perm, 128, tiles, xg, bhist, ctl, s,
+    if ((st = launch_route(L, x, T, logits, ids, w, sgate, counts, offsets, perm, 128, tiles, xg, bhist, ctl, s,
                            launches)) != REDMOE_OK)
         return st;
     if (dbg) {

@@ -2,9 +2,8 @@
 // per SM, each block owning a contiguous range of tokens:
 //
 //   phase 1  one warp per token: top-k of the logits (ties to the lower id) with the
-//            renormalised weights, the shared gate sigmoid(x . g) and a zeroed output row
-//            (the down projection adds into it); the block's histogram of expert ids
-//            goes to bhist[block][e]
+//            renormalised weights and the shared gate sigmoid(x . g); the block's
+//            histogram of expert ids goes to bhist[block][e]
 //   phase 2  per expert e: exclusive prefix of bhist[.][e] over the blocks, and counts[e]
 //   phase 3  per block: the exclusive prefix of the counts (offsets, and block 0 writes
 //            offsets and the GEMM tile schedule), then the block's rows in (t, j) order:
@@ -38,7 +37,6 @@ struct RouteParams {
     int32_t* ids;         // [T, k]
     float* w;             // [T, k]
     float* sgate;         // [T]
-    float* out;           // [T, H] zeroed here
     int32_t* counts;      // [E]
     int32_t* offsets;     // [E + 1]
     int32_t* perm;        // [T * k]
@@ -94,7 +92,8 @@ __global__ void __launch_bounds__(RT_THREADS, 1) route_kernel(const __grid_const
     int* offs = hist + E;            // [E + 1]
     int* tmp = offs + E + 1;         // [E]
     int* wsum = tmp + E;             // [RT_WARPS + 1]
-    int* s_pos = wsum + 32;          // [tpb * k] positions of this block's rows
+    int* s_ids = wsum + 32;          // [tpb * k] this block's expert ids
+    int* s_pos = s_ids + p.tpb * k;  // [tpb * k] positions of this block's rows
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const unsigned nb = gridDim.x;
     const int t0 = min(T, int(blockIdx.x) * p.tpb), t1 = min(T, t0 + p.tpb);
@@ -103,6 +102,18 @@ __global__ void __launch_bounds__(RT_THREADS, 1) route_kernel(const __grid_const
     __syncthreads();
     // ------------------------------------------------------------------ phase 1
     for (int t = t0 + warp; t < t1; t += RT_WARPS) {
+        // the shared gate's first 2048 elements (16-byte loads, eight per lane) and the
+        // logits are loaded together, so the top-k and the dot share one memory latency
+        const uint4* xr = reinterpret_cast<const uint4*>(p.x + size_t(t) * p.H);
+        const uint4* gr = reinterpret_cast<const uint4*>(p.g);
+        const int nc = p.H / 8;
+        uint4 xv[8], gv[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const int c = 32 * i + lane;
+            xv[i] = c < nc ? __ldg(xr + c) : make_uint4(0u, 0u, 0u, 0u);
+            gv[i] = c < nc ? __ldg(gr + c) : make_uint4(0u, 0u, 0u, 0u);
+        }
         uint32_t key[EPL];
         const float* lr = p.logits + size_t(t) * E;
 #pragma unroll
@@ -113,20 +124,18 @@ __global__ void __launch_bounds__(RT_THREADS, 1) route_kernel(const __grid_const
         if (lane < k) {
             p.ids[size_t(t) * k + lane] = id;
             p.w[size_t(t) * k + lane] = wv;
+            s_ids[(t - t0) * k + lane] = id;
             atomicAdd(&hist[id], 1);
         }
-        // shared gate: 16-byte loads, eight chunks of 8 elements per lane issued together
-        const uint4* xr = reinterpret_cast<const uint4*>(p.x + size_t(t) * p.H);
-        const uint4* gr = reinterpret_cast<const uint4*>(p.g);
-        const int nc = p.H / 8;
         float acc = 0.0f;
         for (int c0 = 0; c0 < nc; c0 += 32 * 8) {
-            uint4 xv[8], gv[8];
+            if (c0 > 0) {
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                const int c = c0 + 32 * i + lane;
-                xv[i] = c < nc ? __ldg(xr + c) : make_uint4(0u, 0u, 0u, 0u);
-                gv[i] = c < nc ? __ldg(gr + c) : make_uint4(0u, 0u, 0u, 0u);
+                for (int i = 0; i < 8; ++i) {
+                    const int c = c0 + 32 * i + lane;
+                    xv[i] = c < nc ? __ldg(xr + c) : make_uint4(0u, 0u, 0u, 0u);
+                    gv[i] = c < nc ? __ldg(gr + c) : make_uint4(0u, 0u, 0u, 0u);
+                }
             }
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
@@ -141,8 +150,6 @@ __global__ void __launch_bounds__(RT_THREADS, 1) route_kernel(const __grid_const
         }
         acc = warp_sum(acc);
         if (lane == 0) p.sgate[t] = 1.0f / (1.0f + expf(-acc));
-        float4* o = reinterpret_cast<float4*>(p.out + size_t(t) * p.H);
-        for (int i = lane; i < p.H / 4; i += 32) o[i] = make_float4(0.f, 0.f, 0.f, 0.f);
     }
     __syncthreads();
     for (int e = threadIdx.x; e < E; e += RT_THREADS) p.bhist[size_t(blockIdx.x) * E + e] = hist[e];
@@ -150,10 +157,17 @@ __global__ void __launch_bounds__(RT_THREADS, 1) route_kernel(const __grid_const
 
     // ------------------------------------------------------------------ phase 2
     for (int e = int(blockIdx.x) * RT_WARPS + warp; e < E; e += int(nb) * RT_WARPS) {
+        int vb[ROUTE_MAX_BLOCKS / 32];  // this expert's count in block 32 c + lane, loaded together
+#pragma unroll
+        for (int c = 0; c < ROUTE_MAX_BLOCKS / 32; ++c) {
+            const int b = 32 * c + lane;
+            vb[c] = b < int(nb) ? __ldcg(p.bhist + size_t(b) * E + e) : 0;
+        }
         int carry = 0;
-        for (int b0 = 0; b0 < int(nb); b0 += 32) {
-            const int b = b0 + lane;
-            const int v = b < int(nb) ? __ldcg(p.bhist + size_t(b) * E + e) : 0;
+#pragma unroll
+        for (int c = 0; c < ROUTE_MAX_BLOCKS / 32; ++c) {
+            const int b = 32 * c + lane;
+            const int v = vb[c];
             int inc = v;
 #pragma unroll
             for (int o = 1; o < 32; o <<= 1) {
@@ -194,7 +208,7 @@ __global__ void __launch_bounds__(RT_THREADS, 1) route_kernel(const __grid_const
         for (int base = t0 * k; base < t1 * k; base += 32) {
             const int i = base + lane;
             const bool ok = i < t1 * k;
-            const int e = ok ? __ldcg(p.ids + i) : -1;
+            const int e = ok ? s_ids[i - t0 * k] : -1;
             const unsigned peers = __match_any_sync(FULL, e);
             if (ok) {
                 const int pos = hist[e] + __popc(peers & lt);
@@ -207,24 +221,47 @@ __global__ void __launch_bounds__(RT_THREADS, 1) route_kernel(const __grid_const
         }
     }
     __syncthreads();
-    // gather: x[t] -> xg[position of (t, j)], one warp per row, 16-byte copies
+    // gather: x[t] -> xg[position of (t, j)]; each warp copies two rows at a time in 16-byte
+    // chunks, every load of both rows issued before their stores
     const int nent = (t1 - t0) * k;
     const int row16 = p.H / 8;
-    for (int j = warp; j < nent; j += RT_WARPS) {
-        const uint4* src = reinterpret_cast<const uint4*>(p.x) + size_t(t0 + j / k) * row16;
-        uint4* dst = reinterpret_cast<uint4*>(p.xg) + size_t(s_pos[j]) * row16;
-#pragma unroll 4
-        for (int c = lane; c < row16; c += 32) dst[c] = __ldg(src + c);
+    const uint4* xs = reinterpret_cast<const uint4*>(p.x);
+    uint4* xd = reinterpret_cast<uint4*>(p.xg);
+    const uint4 z4 = make_uint4(0u, 0u, 0u, 0u);
+    for (int j0 = 2 * warp; j0 < nent; j0 += 2 * RT_WARPS) {
+        const int j1 = j0 + 1;
+        const bool two = j1 < nent;
+        const uint4* s0 = xs + size_t(t0 + j0 / k) * row16;
+        const uint4* s1 = xs + size_t(t0 + (two ? j1 : j0) / k) * row16;
+        uint4* d0 = xd + size_t(s_pos[j0]) * row16;
+        uint4* d1 = xd + size_t(s_pos[two ? j1 : j0]) * row16;
+        for (int c0 = 0; c0 < row16; c0 += 32 * 8) {
+            uint4 a[8], b[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const int c = c0 + 32 * i + lane;
+                a[i] = c < row16 ? __ldg(s0 + c) : z4;
+                b[i] = (two && c < row16) ? __ldg(s1 + c) : z4;
+            }
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const int c = c0 + 32 * i + lane;
+                if (c < row16) {
+                    d0[c] = a[i];
+                    if (two) d1[c] = b[i];
+                }
+            }
+        }
     }
     grid_exit(p.ctl, nb);
 }
 
-int route_smem_bytes(int E, int tpb, int k) { return 4 * (3 * E + 1 + 32 + tpb * k); }
+int route_smem_bytes(int E, int tpb, int k) { return 4 * (3 * E + 1 + 32 + 2 * tpb * k); }
 
 }  // namespace
 
 redmoe_status launch_route(const redmoe_layer* L, const void* x, int T, const float* logits, int32_t* ids, float* w,
-                           float* sgate, float* out, int32_t* counts, int32_t* offsets, int32_t* perm, int tile_m,
+                           float* sgate, int32_t* counts, int32_t* offsets, int32_t* perm, int tile_m,
                            int32_t* tiles, void* xg, int32_t* bhist, Control* ctl, cudaStream_t stream,
                            int* launches) {
     DevInfo di;
@@ -237,7 +274,7 @@ redmoe_status launch_route(const redmoe_layer* L, const void* x, int T, const fl
     p.g = static_cast<const uint16_t*>(L->shared_gate_w);
     p.T = T; p.E = E; p.k = k; p.H = L->hidden;
     p.tpb = (T + nb - 1) / nb;
-    p.ids = ids; p.w = w; p.sgate = sgate; p.out = out;
+    p.ids = ids; p.w = w; p.sgate = sgate;
     p.counts = counts; p.offsets = offsets; p.perm = perm; p.tile_m = tile_m; p.tiles = tiles;
     p.xg = static_cast<uint16_t*>(xg); p.bhist = bhist; p.ctl = ctl; p.timeout_ns = BARRIER_TIMEOUT_NS;
     const int smem = route_smem_bytes(E, p.tpb, k);
