@@ -100,21 +100,29 @@ def layer_call_bytes(shape, T, distinct):
             + T * shape.H * xb + T * shape.H * 4 + T * shape.k * 8)
 
 
-def source_digest(kernel_file):
+# kernel sources behind each path: a committed DRAM-traffic figure stays valid while these
+# files are unchanged
+DECODE_SOURCES = ["common.cuh", "decode.cu", "gemv.cuh", "internal.h", "topk.cuh"]
+PREFILL_SOURCES = ["common.cuh", "ggemm.cu", "ggemm_params.h", "internal.h", "prefill.cu", "route.cu", "tc.cuh", "topk.cuh"]
+
+
+def source_digest(files):
     h = hashlib.sha256()
-    for f in sorted(os.listdir(os.path.join(ROOT, "sparse_moe_gemv_b200", "csrc"))):
-        if f.endswith((".cu", ".cuh", ".h")):
-            h.update(open(os.path.join(ROOT, "sparse_moe_gemv_b200", "csrc", f), "rb").read())
+    for f in sorted(files):
+        h.update(f.encode())
+        h.update(open(os.path.join(ROOT, "sparse_moe_gemv_b200", "csrc", f), "rb").read())
     return h.hexdigest()[:16]
 
 
 def profile_traffic(workload):
-    """DRAM bytes per launch from the committed ncu summary, if it matches this source."""
+    """DRAM bytes per launch (per step for the batched layer) from the committed ncu summary,
+    if it was taken on the current kernel sources."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
         return None
     d = json.load(open(p)).get(workload)
-    if not d or d.get("source_digest") != source_digest(None):
+    files = PREFILL_SOURCES if workload == "prefill" else DECODE_SOURCES
+    if not d or d.get("source_digest") != source_digest(files):
         return None
     return d.get("dram_bytes_per_launch")
 
