@@ -127,7 +127,7 @@ redmoe_status redmoe_workspace_init(void *workspace, size_t workspace_bytes, voi
  * the grouping, and tensor-core grouped GEMMs for the experts (gate/up with SwiGLU,
  * then down with a weighted fp32 scatter-add into out, whose summation order is not
  * fixed). The batched path needs bf16 x, router and experts, shared_inter == inter,
- * hidden % 256 == 0, inter % 128 == 0 and inter <= 512; other layers at T > 4 return
+ * hidden % 256 == 0 and inter % 128 == 0; other layers at T > 4 return
  * REDMOE_ERR_UNSUPPORTED. */
 redmoe_status redmoe_forward(const redmoe_layer *L, const void *x, int32_t T, float *out,
                              int32_t *topk_ids, float *topk_w, void *workspace,

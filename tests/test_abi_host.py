@@ -147,3 +147,25 @@ def test_noalloc_rejects_before_touching_cuda(lib):
     # a layer whose decode scratch exceeds the fixed 1 MiB array is refused
     big = _layer(top_k=32, inter=2048, n_experts=64)
     assert f(C.byref(big), FAKE, 4, FAKE, FAKE, FAKE, 0) == WORKSPACE
+
+
+def test_batched_path_shape_rules(lib):
+    """T > 4 runs the batched path, which takes bf16 layers with shared_inter == inter,
+    hidden % 256 == 0 and inter % 128 == 0; the others are refused on the host before any
+    CUDA call."""
+    sc = {n: FAKE + 0x10000000 + 0x100000 * i for i, n in
+          enumerate(("s_gate", "s_up", "s_down", "sh_s_gate", "sh_s_up", "sh_s_down"))}
+    assert _fwd(lib, _layer(expert_dtype=2, **sc), T=8) == UNSUPPORTED          # int4 experts
+    assert _fwd(lib, _layer(shared_inter=256), T=8) == UNSUPPORTED              # shared_inter != inter
+    assert _fwd(lib, _layer(inter=96, shared_inter=96), T=8) == UNSUPPORTED     # inter % 128 != 0
+    assert _fwd(lib, _layer(hidden=2080), T=8) == UNSUPPORTED                   # hidden % 256 != 0
+    assert _fwd(lib, _layer(x_dtype=0, router_dtype=0, expert_dtype=0), T=8) == UNSUPPORTED  # fp32 layer
+
+
+def test_batched_workspace_holds_the_grouped_buffers(lib):
+    L = _layer()
+    T, k, H, I, E = 2048, 10, 2048, 512, 512
+    need = lib.redmoe_workspace_bytes(C.byref(L), T)
+    # logits, the gathered x rows and the SwiGLU rows at least
+    assert need >= 4 * T * E + 2 * T * k * H + 2 * (T * k + T) * I
+    assert need % 256 == 0
