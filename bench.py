@@ -267,8 +267,11 @@ def reference_arm(args, wl, world, rank):
         for l in range(wl["layers"] if wl["stack"] else 1):
             oracle.forward(layers[(s + l) % nl], shape, xs[s % 4])
 
-    for s in range(args.warmup):
+    tw = time.perf_counter()
+    for s in range(args.warmup):  # warm-up, bounded in time like the timed loop
         step(s)
+        if time.perf_counter() - tw > 30.0:
+            break
     budget = 120.0
     t0 = time.perf_counter()
     done = 0
