@@ -16,8 +16,10 @@
 //      combine happens in registers, deterministically, with no atomics).
 //
 // Weight bytes move with 1-D bulk copies (cp.async.bulk, completion on an mbarrier): each
-// warp owns a ring of 3-4 stages of 4 KiB and keeps all but one of them in flight while it
-// computes on the oldest, so a few instructions keep ~100 KB per SM in flight. Compute
+// warp owns a ring of 3-5 stages of 4 KiB (phases A and B add the stages that fit the h
+// buffer, idle until phase C) and keeps them in flight while it computes on the oldest, so
+// a few instructions keep 100-200 KB per SM in flight. bf16 activations are widened to fp32
+// in shared memory once per layer (T <= 3) for the dots. Compute
 // reads the staged rows from shared memory with conflict-free 16-byte accesses ("pieces":
 // 16 bytes of activations and the weight bytes that multiply them), in short rolled
 // loops: at this size the cost is latency and instruction fetch, not arithmetic. The first
@@ -49,7 +51,10 @@ constexpr int RQ_MAX = 8;       // phase-C rows per stage, at most
 constexpr int MAX_SLOTS = DECODE_MAX_T * MAX_TOPK;
 static_assert(MAX_SLOTS <= THREADS, "one thread per routed slot");
 
+// Stages per warp ring in phase C; phases A and B add the stages that fit the h buffer,
+// which is idle until phase C (up to NS_MAX).
 template <int T> struct Stages { static constexpr int NS = (T == 1) ? 5 : ((T == 2) ? 4 : 3); };
+constexpr int NS_MAX = 8;
 
 __host__ __device__ constexpr int align16(int x) { return (x + 15) & ~15; }
 __host__ __device__ constexpr int align128(int x) { return (x + 127) & ~127; }
@@ -57,16 +62,30 @@ __host__ __device__ constexpr int align128(int x) { return (x + 127) & ~127; }
 __host__ __device__ constexpr int scale_bytes(int wt, int K) { return wt == DT_INT4 ? K / 16 : 0; }
 
 struct Smem {
-    int ring, xs, hs, bars, keys, ids, wts, first, uidx, wcnt, ue, umask, uslot, uw, sg, nu, part, jobq, total;
+    int ring, xs, xf, hs, bars, keys, ids, wts, first, uidx, wcnt, ue, umask, uslot, uw, sg, nu, part, jobq, total;
+    int nsb;  // ring depth of phases A and B
 };
 
-__host__ __device__ inline Smem smem_layout(int T, int NS, int H, int E, int k, int I, int Is, int xt, int RB) {
+// bf16 activations are widened to fp32 once per layer (xf) when T <= 3, so that the many
+// weight rows dotted with them do not each convert them again; at T = 4 the fp32 copy does
+// not fit next to the stage ring, and the dots read the bf16 activations.
+template <int XT, int T>
+struct XWide {
+    static constexpr bool on = XT == DT_BF16 && T <= 3;
+    static constexpr int vt = on ? DT_F32 : XT;  // activation type the dots read
+};
+
+__host__ __device__ inline Smem smem_layout(int T, int NS, int H, int E, int k, int I, int Is, int xt, int RB,
+                                            bool xwide) {
     Smem s;
     int o = 0;
     s.ring = o; o += WARPS * NS * SB;
     s.xs = o; o = align128(o + T * H * vbytes(xt));
+    s.xf = o; o = align128(o + (xwide ? T * H * 4 : 0));
     s.hs = o; o = align128(o + 4 * (T * k * I + T * Is));
-    s.bars = o; o += 8 * (WARPS * NS + 2);
+    s.nsb = NS + (4 * (T * k * I + T * Is)) / (WARPS * SB);
+    if (s.nsb > NS_MAX) s.nsb = NS_MAX;
+    s.bars = o; o += 8 * (WARPS * NS_MAX + 2);
     // phase-B scratch (keys, first) and phase-C scratch (part) share one region
     s.keys = o;
     s.first = o + 4 * T * E;
@@ -174,39 +193,47 @@ __device__ __forceinline__ void seg_add(Seg& s, const void* src, uint32_t bytes,
     ++s.n;
 }
 
-// A warp-private ring of NS stages. Lane 0 issues the bulk copies of a stage; every lane
-// waits on the stage's mbarrier; the stage is refilled only after the warp has finished
-// reading it (__syncwarp, then a proxy fence before the async-proxy write).
-template <int NS>
+// A warp-private ring of stages. Lane 0 issues the bulk copies of a stage; every lane waits
+// on the stage's mbarrier; the stage is refilled only after the warp has finished reading it
+// (__syncwarp, then a proxy fence before the async-proxy write). Stages 0 .. nsc-1 live in
+// the ring region, the others in the h buffer; the depth may change only when the ring is
+// drained. Each stage's next completion parity is one bit of `phase`.
 struct Ring {
-    unsigned char* buf;
+    unsigned char* buf0;  // stages 0 .. nsc-1
+    unsigned char* buf1;  // stages nsc .. (h buffer)
     uint64_t* bar;
-    uint32_t issued, consumed;
+    uint32_t issued, consumed, phase;
+    int ns, nsc, si, sc;  // depth, ring-region depth, next stage to issue, next to consume
 
+    __device__ __forceinline__ unsigned char* stage(int st) const { return st < nsc ? buf0 + st * SB : buf1 + (st - nsc) * SB; }
     __device__ __forceinline__ void issue(const Seg& s, int lane) {
-        const int st = int(issued % NS);
+        const int st = si;
         if (lane == 0) {
             fence_proxy_async_smem();
             uint32_t tot = 0;
 #pragma unroll
             for (int i = 0; i < 4; ++i) tot += (i < s.n) ? s.bytes[i] : 0u;
             mbar_arrive_expect_tx(bar + st, tot);
+            unsigned char* dst = stage(st);
 #pragma unroll
             for (int i = 0; i < 4; ++i)
-                if (i < s.n) bulk_g2s(buf + st * SB + s.off[i], s.src[i], s.bytes[i], bar + st);
+                if (i < s.n) bulk_g2s(dst + s.off[i], s.src[i], s.bytes[i], bar + st);
         }
+        si = (si + 1 == ns) ? 0 : si + 1;
         ++issued;
     }
     __device__ __forceinline__ const unsigned char* wait(int* err, uint64_t timeout_ns) {
-        const int st = int(consumed % NS);
-        mbar_wait(bar + st, (consumed / NS) & 1u, err, timeout_ns);
-        return buf + st * SB;
+        mbar_wait(bar + sc, (phase >> sc) & 1u, err, timeout_ns);
+        return stage(sc);
     }
     __device__ __forceinline__ void release() {
         __syncwarp();
+        phase ^= 1u << sc;
+        sc = (sc + 1 == ns) ? 0 : sc + 1;
         ++consumed;
     }
-    __device__ __forceinline__ bool full() const { return issued - consumed >= uint32_t(NS); }
+    __device__ __forceinline__ bool full() const { return issued - consumed >= uint32_t(ns); }
+    __device__ __forceinline__ void set_depth(int n) { ns = n; si = sc = 0; }  // drained rings only
 };
 
 template <int NL>
@@ -234,11 +261,12 @@ __global__ void __launch_bounds__(THREADS, 1) decode_kernel(const __grid_constan
     const int Wtot = nblocks * WARPS;
     int* err = &p.ctl->err;
     const uint64_t to = p.timeout_ns;
-    const Smem S = smem_layout(T, NS, H, E, k, I, Is, XT, p.RB);
+    using XW = XWide<XT, T>;
+    const Smem S = smem_layout(T, NS, H, E, k, I, Is, XT, p.RB, XW::on);
     unsigned char* xs = smem + S.xs;
     unsigned char* hs = smem + S.hs;
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S.bars);
-    uint64_t* xbar = bars + WARPS * NS;
+    uint64_t* xbar = bars + WARPS * NS_MAX;
     uint64_t* hbar = xbar + 1;
     uint32_t* s_keys = reinterpret_cast<uint32_t*>(smem + S.keys);
     int* s_ids = reinterpret_cast<int*>(smem + S.ids);
@@ -255,12 +283,15 @@ __global__ void __launch_bounds__(THREADS, 1) decode_kernel(const __grid_constan
     float* s_part = reinterpret_cast<float*>(smem + S.part);
     int* s_jobq = reinterpret_cast<int*>(smem + S.jobq) + warp * 8;  // job code of each ring stage
 
-    Ring<NS> ring;
-    ring.buf = smem + S.ring + warp * NS * SB;
-    ring.bar = bars + warp * NS;
-    ring.issued = ring.consumed = 0;
+    Ring ring;
+    ring.buf0 = smem + S.ring + warp * NS * SB;
+    ring.buf1 = smem + S.hs + warp * (S.nsb - NS) * SB;
+    ring.bar = bars + warp * NS_MAX;
+    ring.issued = ring.consumed = ring.phase = 0u;
+    ring.nsc = NS;
+    ring.set_depth(S.nsb);
     if (lane == 0)
-        for (int i = 0; i < NS; ++i) mbar_init(ring.bar + i, 1);
+        for (int i = 0; i < NS_MAX; ++i) mbar_init(ring.bar + i, 1);
     if (threadIdx.x == 0) {
         mbar_init(xbar, 1);
         mbar_init(hbar, 1);
@@ -269,6 +300,8 @@ __global__ void __launch_bounds__(THREADS, 1) decode_kernel(const __grid_constan
     __syncthreads();
 
     const int xrow = H * vbytes(XT);                 // bytes of one activation row
+    const unsigned char* xv = XW::on ? smem + S.xf : xs;  // activations as the dots read them
+    const int xvrow = XW::on ? H * 4 : xrow;
     const int rrow = int(row_bytes(RT, H));          // router / shared-gate row
     const int grow = int(row_bytes(WT, H));          // gate or up row
     const int gsc = scale_bytes(WT, H);
@@ -300,6 +333,7 @@ __global__ void __launch_bounds__(THREADS, 1) decode_kernel(const __grid_constan
         const char* sh_gate = static_cast<const char*>(Ly.sh_gate);
         const char* sh_up = static_cast<const char*>(Ly.sh_up);
 
+        ring.set_depth(S.nsb);  // drained: phases A and B borrow the h buffer
         // ---------------------------------------------------------- phase A
         // Router rows 0..E-1 and the shared gate row (job E), by warps 1..7 of every block
         // (warp 0 only starts copies of its phase-B rows).
@@ -339,7 +373,7 @@ __global__ void __launch_bounds__(THREADS, 1) decode_kernel(const __grid_constan
                 bcur = bj;
                 bj += Wtot;
             }
-            if (lane == 0) s_jobq[ring.issued % NS] = (bcur << 1) | bp;
+            if (lane == 0) s_jobq[ring.si] = (bcur << 1) | bp;
             ring.issue(segB(bcur, bp, Ucur), lane);
             if (++bp == pparts) bp = 0;
             return true;
@@ -359,12 +393,18 @@ __global__ void __launch_bounds__(THREADS, 1) decode_kernel(const __grid_constan
             while (!ring.full() && aj < jobsA) { ring.issue(segA(aj), lane); aj += WA; }
             while (!ring.full() && aj >= jobsA && issueB()) {}  // shared gate/up copies ahead of routing
             mbar_wait(xbar, l & 1, err, to);
+            if (XW::on) {  // widen this layer's activations once
+                const uint32_t* x2 = reinterpret_cast<const uint32_t*>(xs);
+                float2* xw = reinterpret_cast<float2*>(smem + S.xf);
+                for (int i = threadIdx.x; i < T * H / 2; i += THREADS) xw[i] = bf2(x2[i]);
+                __syncthreads();
+            }
             for (int job = wA; job < jobsA; job += WA) {
                 float2 a[T];
 #pragma unroll
                 for (int t = 0; t < T; ++t) a[t] = make_float2(0.f, 0.f);
                 const unsigned char* d = ring.wait(err, to);
-                staged_dot<RT, XT, T>(d, nullptr, H, xs, xrow, lane, a);
+                staged_dot<RT, XW::vt, T>(d, nullptr, H, xv, xvrow, lane, a);
                 ring.release();
                 if (aj < jobsA) {
                     ring.issue(segA(aj), lane);
@@ -488,13 +528,13 @@ __global__ void __launch_bounds__(THREADS, 1) decode_kernel(const __grid_constan
 #pragma unroll
             for (int t = 0; t < T; ++t) a[t] = b[t] = make_float2(0.f, 0.f);
             while (ring.consumed != ring.issued) {
-                const int code = s_jobq[ring.consumed % NS];
+                const int code = s_jobq[ring.sc];
                 const int job = code >> 1, part = code & 1;
                 const unsigned char* d = ring.wait(err, to);
-                if (pair1 || part == 0) staged_dot<WT, XT, T>(d, d + align16(grow), H, xs, xrow, lane, a);
+                if (pair1 || part == 0) staged_dot<WT, XW::vt, T>(d, d + align16(grow), H, xv, xvrow, lane, a);
                 if (pair1 || part == 1) {
                     const unsigned char* du = d + (pair1 ? gtot : 0);
-                    staged_dot<WT, XT, T>(du, du + align16(grow), H, xs, xrow, lane, b);
+                    staged_dot<WT, XW::vt, T>(du, du + align16(grow), H, xv, xvrow, lane, b);
                 }
                 ring.release();
                 issueB();
@@ -523,6 +563,7 @@ __global__ void __launch_bounds__(THREADS, 1) decode_kernel(const __grid_constan
         grid_arrive(p.ctl);
         int cj = cgrp;  // issue cursor of phase C (expert slot)
         const bool has_rows = cq * rq < nrows;
+        ring.set_depth(NS);  // drained: phase C keeps the h buffer for h
         while (has_rows && !ring.full() && cj < jobsC) { ring.issue(segC(cj), lane); cj += gpc; }
         grid_wait(p.ctl, nblocks, bar_idx++, to);
 
@@ -660,7 +701,8 @@ redmoe_status launch_one(const redmoe_layer* sh, const DecLayer* layers, int n_l
     const int RB = (sh->hidden + di.sm_count - 1) / di.sm_count;
     const int RQ = decode_rows_per_stage(sh);
     if (RQ < 1 || RB > WARPS * RQ) return REDMOE_ERR_UNSUPPORTED;
-    const Smem S = smem_layout(T, Stages<T>::NS, sh->hidden, sh->n_experts, sh->top_k, sh->inter, sh->shared_inter, XT, RB);
+    const Smem S = smem_layout(T, Stages<T>::NS, sh->hidden, sh->n_experts, sh->top_k, sh->inter, sh->shared_inter, XT, RB,
+                               XWide<XT, T>::on);
     if (S.total > di.max_smem_optin) return REDMOE_ERR_UNSUPPORTED;
     auto kern = decode_kernel<XT, RT, WT, T, NL>;
     const int per_sm = blocks_per_sm(reinterpret_cast<const void*>(kern), S.total);
