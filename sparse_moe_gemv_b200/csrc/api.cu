@@ -11,8 +11,7 @@
 namespace redmoe {
 
 redmoe_status launch_router(const redmoe_layer* L, const void* x, int T, float* logits, int32_t* ids, float* w,
-                            float* sgate, float* zero_out, bool compute_logits, cudaStream_t stream,
-                            int* launches);
+                            float* sgate, cudaStream_t stream, int* launches);
 redmoe_status launch_route_build(const int32_t* ids, int T, int k, int E, int32_t* counts, int32_t* offsets,
                                  int32_t* perm, int tile_m, int32_t* tiles, cudaStream_t stream, int* launches);
 int route_build_smem_bytes(int E);
@@ -208,7 +207,7 @@ redmoe_status redmoe_router(const redmoe_layer* L, const void* x, int32_t T, int
     if ((st = check_ws(L, T, workspace, workspace_bytes)) != REDMOE_OK) return st;
     const BatchWs b = batch_ws_layout(T, L->n_experts);
     float* lg = logits ? logits : reinterpret_cast<float*>(static_cast<char*>(workspace) + b.logits);
-    return launch_router(L, x, T, lg, topk_ids, topk_w, shared_gate, nullptr, true,
+    return launch_router(L, x, T, lg, topk_ids, topk_w, shared_gate,
                          static_cast<cudaStream_t>(stream), nullptr);
 }
 

@@ -1,14 +1,12 @@
-// Router stage for any number of token rows (the batched path and redmoe_router):
+// Router stage of redmoe_router, for any number of token rows:
 //   router_logits_kernel  l[t, e] = x_t . Wr[e] (+ b[e])   (CUDA cores, rows streamed once
-//                         per block of 4 tokens; the prefill path computes the same logits
-//                         with the tensor-core GEMM instead)
+//                         per block of 4 tokens; the batched forward path computes the same
+//                         logits with a tensor-core GEMM and its top-k in route.cu)
 //   topk_kernel           per token (one warp): top-k of the logits with ties to the lower
-//                         id, renormalised weights, shared gate sigmoid(x . g), and
-//                         optionally a zeroed output row for the scatter-add combine.
+//                         id, renormalised weights and the shared gate sigmoid(x . g).
 // Router, top-k and shared gate belong to one stage of the layer ("Research notes,
 // October 2026", section 1 "DwarfStar today": router, top-k and shared gate run in one
-// kernel); here the logits of a large batch come from a GEMM, so the top-k and gate
-// run as the epilogue kernel that follows it.
+// kernel).
 #include "common.cuh"
 #include "gemv.cuh"
 #include "internal.h"
@@ -58,7 +56,7 @@ __global__ void __launch_bounds__(RL_THREADS) router_logits_kernel(const void* x
 template <int XT, int RT>
 __global__ void __launch_bounds__(RL_THREADS) topk_kernel(const float* logits, int T, int E, int k, const void* x,
                                                           const void* g, int H, int32_t* ids, float* w,
-                                                          float* sgate, float* zero_out) {
+                                                          float* sgate) {
     extern __shared__ __align__(16) uint32_t keys[];  // [RL_WARPS][E]
     const int lane = threadIdx.x & 31;
     const int t = blockIdx.x * RL_WARPS + (threadIdx.x >> 5);
@@ -101,34 +99,27 @@ __global__ void __launch_bounds__(RL_THREADS) topk_kernel(const float* logits, i
     }
     acc = warp_sum(acc);
     if (lane == 0 && sgate) sgate[t] = 1.0f / (1.0f + expf(-acc));
-    if (zero_out) {
-        float4* o = reinterpret_cast<float4*>(zero_out + size_t(t) * H);
-        for (int i = lane; i < H / 4; i += 32) o[i] = make_float4(0.f, 0.f, 0.f, 0.f);
-    }
 }
 
 template <int XT, int RT>
 redmoe_status launch_router_dt(const redmoe_layer* L, const void* x, int T, float* logits, int32_t* ids,
-                               float* w, float* sgate, float* zero_out, bool compute_logits,
-                               cudaStream_t stream, int* launches) {
+                               float* w, float* sgate, cudaStream_t stream, int* launches) {
     const int H = L->hidden, E = L->n_experts;
-    if (compute_logits) {
-        const int smem = RL_TOK * staged_bytes(H, RT, XT);
-        auto kern = router_logits_kernel<XT, RT>;
-        if (smem > 48 * 1024 &&
-            cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
-            return REDMOE_ERR_CUDA;
-        dim3 grid((E + RL_WARPS - 1) / RL_WARPS, (T + RL_TOK - 1) / RL_TOK);
-        kern<<<grid, RL_THREADS, smem, stream>>>(x, T, H, E, L->router_w, L->router_bias, logits);
-        if (cudaGetLastError() != cudaSuccess) return REDMOE_ERR_CUDA;
-        if (launches) *launches += 1;
-    }
+    const int smem = RL_TOK * staged_bytes(H, RT, XT);
+    auto kern = router_logits_kernel<XT, RT>;
+    if (smem > 48 * 1024 &&
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+        return REDMOE_ERR_CUDA;
+    dim3 grid((E + RL_WARPS - 1) / RL_WARPS, (T + RL_TOK - 1) / RL_TOK);
+    kern<<<grid, RL_THREADS, smem, stream>>>(x, T, H, E, L->router_w, L->router_bias, logits);
+    if (cudaGetLastError() != cudaSuccess) return REDMOE_ERR_CUDA;
+    if (launches) *launches += 1;
     const int ksmem = RL_WARPS * E * 4;
     if (ksmem > 48 * 1024 &&
         cudaFuncSetAttribute(topk_kernel<XT, RT>, cudaFuncAttributeMaxDynamicSharedMemorySize, ksmem) != cudaSuccess)
         return REDMOE_ERR_CUDA;
     topk_kernel<XT, RT><<<(T + RL_WARPS - 1) / RL_WARPS, RL_THREADS, ksmem, stream>>>(
-        logits, T, E, L->top_k, x, L->shared_gate_w, H, ids, w, sgate, zero_out);
+        logits, T, E, L->top_k, x, L->shared_gate_w, H, ids, w, sgate);
     if (cudaGetLastError() != cudaSuccess) return REDMOE_ERR_CUDA;
     if (launches) *launches += 1;
     return REDMOE_OK;
@@ -137,12 +128,11 @@ redmoe_status launch_router_dt(const redmoe_layer* L, const void* x, int T, floa
 }  // namespace
 
 redmoe_status launch_router(const redmoe_layer* L, const void* x, int T, float* logits, int32_t* ids, float* w,
-                            float* sgate, float* zero_out, bool compute_logits, cudaStream_t stream,
-                            int* launches) {
+                            float* sgate, cudaStream_t stream, int* launches) {
     if (L->x_dtype == DT_F32 && L->router_dtype == DT_F32)
-        return launch_router_dt<DT_F32, DT_F32>(L, x, T, logits, ids, w, sgate, zero_out, compute_logits, stream, launches);
+        return launch_router_dt<DT_F32, DT_F32>(L, x, T, logits, ids, w, sgate, stream, launches);
     if (L->x_dtype == DT_BF16 && L->router_dtype == DT_BF16)
-        return launch_router_dt<DT_BF16, DT_BF16>(L, x, T, logits, ids, w, sgate, zero_out, compute_logits, stream, launches);
+        return launch_router_dt<DT_BF16, DT_BF16>(L, x, T, logits, ids, w, sgate, stream, launches);
     return REDMOE_ERR_UNSUPPORTED;
 }
 
