@@ -53,7 +53,7 @@ def test_qwen_bf16(gpu_lib, T):
     assert_layer_parity(shape, L, x, out, ids, w, ot, wt, f"bf16 T={T}")
 
 
-@pytest.mark.parametrize("T", [1, 3])
+@pytest.mark.parametrize("T", [1, 2, 3, 4])
 def test_qwen_int4(gpu_lib, T):
     shape = QWEN_INT4
     L = _dev_layer(shape, 4000 + T)

@@ -76,3 +76,63 @@ def test_prefill_chunk_zipf_2048(gpu_lib):
     assert sorted(perm.tolist()) == list(range(T * shape.k))
     # the workload's shape: a few hot experts take hundreds of tokens, most take none
     assert int((c_ref >= 100).sum()) >= 5 and int((c_ref == 0).sum()) >= 200
+
+
+MID = mi.LayerShape(H=512, E=40, k=3, I=256, Is=256, sigma=0.04)
+
+
+@pytest.mark.parametrize("T", [6, 250])
+def test_mid_layer_batched(gpu_lib, T):
+    """Several n-tiles in both grouped GEMMs (I / 128 = 2, H / 256 = 2) and a router width
+    that is not a multiple of the 64-expert GEMM tile."""
+    shape = MID
+    L = mi.make_layer(shape, 500 + T, "cuda")
+    x = mi.make_x(shape, T, 500 + T, "cuda")
+    out, ids, w, _ = _run(shape, L, x)
+    ot, wt = tolerances(shape)
+    assert_layer_parity(shape, L, x, out, ids, w, ot, wt, f"mid batched T={T}")
+
+
+def test_top1_routing_batched(gpu_lib):
+    shape = mi.LayerShape(H=256, E=16, k=1, I=128, Is=128, sigma=0.05)
+    T = 64
+    L = mi.make_layer(shape, 640, "cuda")
+    x = mi.make_x(shape, T, 640, "cuda")
+    out, ids, w, _ = _run(shape, L, x)
+    assert torch.all(w == 1.0)  # renormalising a single selection gives weight 1
+    ot, wt = tolerances(shape)
+    assert_layer_parity(shape, L, x, out, ids, w, ot, wt, "top-1 batched")
+
+
+def test_chunk_4096_all_experts(gpu_lib):
+    """A 4096-token chunk with unbiased routing: every expert receives tokens and every CTA
+    of the grouped GEMMs runs many tiles. Ids and weights of every token, the grouping,
+    and the outputs of a sample of 64 tokens."""
+    shape = QWEN
+    T = 4096
+    L = mi.make_layer(shape, 4096, "cuda")
+    x = mi.make_x(shape, T, 4096, "cuda")
+    out, ids, w, dbg = _run(shape, L, x, dbg=True)
+    rows = np.sort(np.random.default_rng(1).choice(T, 64, replace=False))
+    ot, wt = tolerances(shape)
+    r = assert_layer_parity(shape, L, x, out, ids, w, ot, wt, "chunk 4096", rows=rows)
+    c_ref, o_ref, p_ref = oracle.route_build(r["ref"]["ids"], shape.E)
+    np.testing.assert_array_equal(dbg[0].cpu().numpy(), c_ref)
+    np.testing.assert_array_equal(dbg[1].cpu().numpy(), o_ref)
+    assert int((c_ref > 0).sum()) == shape.E
+
+
+def test_batched_repeat_is_stable(gpu_lib):
+    """Two calls on the same input: ids, weights and grouping are identical; the outputs
+    differ at most by the order of the fp32 reductions of the combine."""
+    shape = QWEN
+    T = 300
+    L = mi.make_layer(shape, 77, "cuda")
+    x = mi.make_x(shape, T, 77, "cuda")
+    o1, i1, w1, d1 = _run(shape, L, x, dbg=True)
+    o2, i2, w2, d2 = _run(shape, L, x, dbg=True)
+    assert torch.equal(i1, i2) and torch.equal(w1, w2)
+    for a, b in zip(d1, d2):
+        assert torch.equal(a, b)
+    scale = float(o1.abs().max())
+    assert float((o1 - o2).abs().max()) <= 1e-5 * scale
