@@ -204,20 +204,27 @@ def barrier(world):
         torch.distributed.barrier()
 
 
-def max_over_ranks(v, world):
+def _reduce(v, world, op):
     if world == 1:
         return v
-    t = torch.tensor([v], dtype=torch.float64, device="cuda")
-    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    # NCCL reduces device tensors; gloo (the CPU tests of this logic) host tensors
+    dev = "cuda" if torch.distributed.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([v], dtype=torch.float64, device=dev)
+    torch.distributed.all_reduce(t, op=op)
     return float(t.item())
+
+
+def max_over_ranks(v, world):
+    return _reduce(v, world, torch.distributed.ReduceOp.MAX)
 
 
 def sum_over_ranks(v, world):
-    if world == 1:
-        return v
-    t = torch.tensor([v], dtype=torch.float64, device="cuda")
-    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.SUM)
-    return float(t.item())
+    return _reduce(v, world, torch.distributed.ReduceOp.SUM)
+
+
+def job_throughput(units, seconds, world):
+    """Whole-job rate: the units every rank processed over the slowest rank's time."""
+    return sum_over_ranks(units, world) / max_over_ranks(seconds, world)
 
 
 # ------------------------------------------------------------- CPU baseline
@@ -371,9 +378,9 @@ def gpu_arm(args, wl, world, rank, local):
     barrier(world)
     smg.redmoe_check_timeout(B["work"], stream=stream)
     el_ms = ev0.elapsed_time(ev1)
-    el_ms = max_over_ranks(el_ms, world)
     tokens_per_step = T * (wl["layers"] if wl["stack"] else 1)
-    value = sum_over_ranks(K * tokens_per_step, world) / (el_ms / 1e3)
+    value = job_throughput(K * tokens_per_step, el_ms / 1e3, world)  # this rank's time in
+    el_ms = max_over_ranks(el_ms, world)
 
     # distinct experts per layer call, from the ids of the last step of each layer
     distinct = []
@@ -465,12 +472,11 @@ def e2e_arm(args, wl, smg, B, stream, world):
             step(i)
     stream.synchronize()
     el = time.perf_counter() - t0
-    el = max_over_ranks(el, world)
     per = (nl if wl["stack"] else 1)
-    tokens = n_e2e * T * per
+    rate = job_throughput(n_e2e * T * per, el, world)  # this rank's wall time in
     h2d = T * shape.H * xb * per
     d2h = (T * shape.H * 4 + T * shape.k * 8) * per
-    return {"value": sum_over_ranks(tokens, world) / el, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+    return {"value": rate, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
             "d2h_bytes_per_step": d2h, "steps": n_e2e,
             "how": "redmoe_forward through the C ABI per step; pinned host x copied in, out/ids/w copied out, "
                    "host wall clock around the K steps"}
