@@ -259,7 +259,8 @@ def reference_arm(args, wl, world, rank):
         return None
     shape = wl["shape"]
     T = wl["T"]
-    cores = oracle.num_threads()
+    threads = oracle.num_threads()
+    cores = min(threads, T)  # the oracle splits a call over its tokens: threads beyond T idle
     nl = min(wl["layers"], 2)
     layers = []
     for l in range(nl):
@@ -292,7 +293,7 @@ def reference_arm(args, wl, world, rank):
     unit = "tokens/s"
     sample = (f"{done} of {args.steps} steps (time-bounded at {budget:.0f} s), each "
               f"{'a ' + str(wl['layers']) + '-layer stack' if wl['stack'] else 'one layer'} at T={T}, "
-              f"fp64 oracle, {cores} threads")
+              f"fp64 oracle, {cores} of {threads} threads busy (OpenMP over the call's tokens)")
     return {"metric": METRIC, "value": value, "unit": unit, "n_gpus": 1, "steps": done, "warmup": args.warmup,
             "ms_per_step": 1e3 * el / max(done, 1), "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
