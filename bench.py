@@ -57,6 +57,10 @@ WORKLOADS = {
                     desc="48 distinct Qwen3-Next-shaped layers, int4 group-32 experts, decode T=1"),
     "prefill": dict(shape=QWEN_ZIPF, T=2048, layers=1, stack=False, seed=3000, kernel="layer (4 kernels)",
                     desc="Qwen3-Next-shaped MoE layer, bf16, 2048-token prefill chunk, Zipf(1.1) router offsets"),
+    # the same chunk with unbiased routing: every expert is touched, so the step streams all
+    # 512 experts' weights and the HBM floor moves above the tensor-core one
+    "prefill_uniform": dict(shape=QWEN, T=2048, layers=1, stack=False, seed=3000, kernel="layer (4 kernels)",
+                            desc="Qwen3-Next-shaped MoE layer, bf16, 2048-token prefill chunk, unbiased router"),
 }
 
 
