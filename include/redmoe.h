@@ -23,7 +23,8 @@
  * Conventions for every entry point:
  *  - Every tensor pointer is DEVICE memory owned by the caller; the library allocates
  *    no memory and keeps no state between calls except a per-device cache of device
- *    attributes. Tensors are dense, row-major, contiguous.
+ *    attributes and the fixed scratch array of redmoe_forward_noalloc (static memory in
+ *    the library image). Tensors are dense, row-major, contiguous.
  *  - `stream` is a cudaStream_t (NULL: the legacy default stream). Work is only
  *    enqueued; no call synchronises the host except redmoe_check_timeout().
  *  - Arguments are validated on the host before anything is enqueued. On any error
