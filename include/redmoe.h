@@ -49,7 +49,7 @@ extern "C" {
 typedef enum {
     REDMOE_OK = 0,
     REDMOE_ERR_INVALID_ARG = 1,   /* null/misaligned pointer, bad size, bad enum value      */
-    REDMOE_ERR_UNSUPPORTED = 2,   /* valid arguments this build has no kernel for           */
+    REDMOE_ERR_UNSUPPORTED = 2,   /* valid arguments the library has no kernel for         */
     REDMOE_ERR_WORKSPACE = 3,     /* workspace null or smaller than redmoe_workspace_bytes  */
     REDMOE_ERR_CUDA = 4,          /* a CUDA runtime call or kernel launch failed            */
     REDMOE_ERR_TIMEOUT = 5        /* a bounded in-kernel wait ran out (see check_timeout)   */
