@@ -169,3 +169,13 @@ def test_batched_workspace_holds_the_grouped_buffers(lib):
     # logits, the gathered x rows and the SwiGLU rows at least
     assert need >= 4 * T * E + 2 * T * k * H + 2 * (T * k + T) * I
     assert need % 256 == 0
+
+
+def test_missing_library_fails_loudly(monkeypatch):
+    """No fallback: without the built library the binding raises, it never computes."""
+    monkeypatch.setattr(smg, "_lib", None)
+    monkeypatch.setattr(smg, "LIB_PATH", os.path.join(os.path.dirname(smg.LIB_PATH), "absent", "libredmoe.so"))
+    with pytest.raises(RuntimeError, match="is missing"):
+        smg.load()
+    with pytest.raises(RuntimeError, match="is missing"):
+        smg.redmoe_status_string(0)
