@@ -27,6 +27,10 @@ MUTANTS = {
     "shared_gate_sign": ("s[t] = 1.0 / (1.0 + exp(-gx));", "s[t] = 1.0 / (1.0 + exp(gx));"),
     "group_order_reversed": ("perm[cursor[ids[i]]++] = (int32_t)i;",
                              "perm[offsets[ids[i] + 1] - 1 - (cursor[ids[i]]++ - offsets[ids[i]])] = (int32_t)i;"),
+    "renorm_not_renormalised": ("w[j] = (exp(logits_row[ids[j]] - m) / z) / ps;",
+                                "w[j] = (exp(logits_row[ids[j]] - m) / z);"),
+    "renorm_wrong_index": ("w[j] = (exp(logits_row[ids[j]] - m) / z) / ps;",
+                           "w[j] = (exp(logits_row[j] - m) / z) / ps;"),
     "scale_group_index": ("double s = bf16_bits_to_double(scale[n * (K / 32) + c / 32]);",
                           "double s = bf16_bits_to_double(scale[n * (K / 32) + (c / 32 + 1) % (K / 32)]);"),
 }

@@ -337,3 +337,42 @@ def test_partial_expert_supply_is_enough_and_missing_is_reported():
     missing["w_down"] = {e: lay["w_down"][e] for e in used[1:]}
     with pytest.raises(oracle.OracleError):
         oracle.forward(missing, shape, x)
+
+
+# ------------------------------------------------------- renormalised subsets
+# oracle.renorm gives the weights of an arbitrary k-subset of one token's experts; the
+# parity checker uses it for tokens on a near-tie, where the valid id set is not unique.
+LOGITS_WORKED = np.log(np.array([1.0, 2.0, 3.0, 4.0]))  # p = (1, 2, 3, 4) / 10
+
+
+@pytest.mark.parametrize("ids,expected", [
+    ((3, 2), (Fraction(4, 7), Fraction(3, 7))),   # the worked example's token 0
+    ((0, 1), (Fraction(1, 3), Fraction(2, 3))),   # a subset the router would not pick
+    ((1, 3), (Fraction(1, 3), Fraction(2, 3))),
+    ((2,), (Fraction(1),)),                      # a single selection renormalises to 1
+    ((0, 1, 2, 3), (Fraction(1, 10), Fraction(2, 10), Fraction(3, 10), Fraction(4, 10))),
+])
+def test_renorm_hand_derived_subsets(ids, expected):
+    w = oracle.renorm(LOGITS_WORKED, np.array(ids, np.int32))
+    np.testing.assert_allclose(w, [float(f) for f in expected], rtol=0, atol=1e-15)
+
+
+def test_renorm_ignores_a_common_logit_shift():
+    # softmax is shift-invariant: p_e / sum_sel p = exp(l_e) / sum_sel exp(l); a shift of
+    # every logit by 700 must not change the weights (nor overflow); l + 700 is stored
+    # with an absolute rounding of up to 2^-44, so the weights agree to about 1e-13
+    ids = np.array([3, 0, 2], np.int32)
+    np.testing.assert_allclose(oracle.renorm(LOGITS_WORKED + 700.0, ids),
+                               [4 / 8, 1 / 8, 3 / 8], rtol=0, atol=1e-12)
+
+
+@pytest.mark.parametrize("name", list(SHAPES))
+def test_renorm_equals_router_weights_for_router_ids(name):
+    shape = SHAPES[name]
+    lay, x = _tiny(shape, 11, T=6)
+    r = oracle.router(lay, shape, x)
+    for t in range(x.shape[0]):
+        np.testing.assert_allclose(oracle.renorm(r["logits"][t], r["ids"][t]), r["w"][t], rtol=0, atol=1e-15)
+        # a reversed order gives the same weights, reversed
+        np.testing.assert_allclose(oracle.renorm(r["logits"][t], r["ids"][t][::-1].copy()), r["w"][t][::-1],
+                                   rtol=0, atol=1e-15)
