@@ -114,7 +114,9 @@ const char *redmoe_status_string(int32_t status);
  * workspace must be ordered on the GPU (same stream or synchronised streams). */
 size_t redmoe_workspace_bytes(const redmoe_layer *L, int32_t T);
 
-/* Zero the control block of a workspace on `stream` (an async memset of 256 bytes). */
+/* Zero the control block of a workspace on `stream` (an async memset of 256 bytes).
+ * workspace == NULL zeroes the control block of the current device's allocation-free
+ * scratch (see redmoe_forward_noalloc) instead; workspace_bytes is then ignored. */
 redmoe_status redmoe_workspace_init(void *workspace, size_t workspace_bytes, void *stream);
 
 /* The whole layer for T token rows.
@@ -146,8 +148,9 @@ redmoe_status redmoe_router(const redmoe_layer *L, const void *x, int32_t T, int
  * counts[e]; perm[offsets[e] + r] = t*k + j for the r-th row (t, j) routed to e in
  * increasing t. Bit-exact and deterministic. The batched path of redmoe_forward uses
  * the same kernel. Out-of-range ids are not detected on the device: they are skipped
- * and the outputs are then unspecified. Workspace: redmoe_workspace_bytes of any layer
- * with these E and k at this T (or at least 256 bytes + 4*(E+1)*ceil(T/64) bytes). */
+ * and the outputs are then unspecified. The kernel needs no scratch memory: workspace
+ * and workspace_bytes are not used (pass NULL and 0); they keep the signature uniform
+ * with the other entry points. */
 redmoe_status redmoe_route_build(const int32_t *topk_ids, int32_t T, int32_t k, int32_t E,
                                  int32_t *counts, int32_t *offsets, int32_t *perm,
                                  void *workspace, size_t workspace_bytes, void *stream);
@@ -172,18 +175,46 @@ redmoe_status redmoe_forward_stack(const redmoe_layer *layers, int32_t n_layers,
  * loads the library holds it until the process exits. Arguments and outputs are those of
  * redmoe_forward. The first call on each device looks up the array's device address
  * (cudaGetSymbolAddress, with that device current): make that first call outside any
- * stream capture. Each call clears the array's control block with an async memset
- * before the kernel; nothing is allocated or freed. All calls on a device share the
- * array, so calls that can overlap on the GPU race and must not be made; order them on
- * one stream. Returns REDMOE_ERR_WORKSPACE if the layer at this T needs more than the
- * 1 MiB scratch, REDMOE_ERR_UNSUPPORTED for T > 4, otherwise as redmoe_forward. */
+ * stream capture. Nothing is allocated or freed. Each call clears the scratch's two
+ * grid-barrier counters with an async 8-byte memset before the kernel; the error word
+ * is kept, so a bounded in-kernel wait that gave up stays visible: read it with
+ * redmoe_check_timeout(NULL, stream) and clear it with redmoe_workspace_init(NULL, 0,
+ * stream); until then later calls may give up their own waits early and their outputs are
+ * unspecified. All calls on a device share the array, so calls that can overlap on the GPU
+ * race and must not be made; order them on one stream. Returns REDMOE_ERR_WORKSPACE if
+ * the layer at this T needs more than the 1 MiB scratch, REDMOE_ERR_UNSUPPORTED for
+ * T > 4, otherwise as redmoe_forward. */
 redmoe_status redmoe_forward_noalloc(const redmoe_layer *L, const void *x, int32_t T, float *out,
                                      int32_t *topk_ids, float *topk_w, void *stream);
 
 /* Synchronise `stream`, then read the workspace's error word: REDMOE_ERR_TIMEOUT if an
  * in-kernel grid barrier gave up waiting (bounded at about one second) since the last
- * redmoe_workspace_init, else REDMOE_OK. REDMOE_ERR_CUDA if the stream reports an error. */
+ * redmoe_workspace_init, else REDMOE_OK. REDMOE_ERR_CUDA if the stream reports an error.
+ * workspace == NULL reads the error word of the current device's allocation-free
+ * scratch (redmoe_forward_noalloc). */
 redmoe_status redmoe_check_timeout(const void *workspace, void *stream);
+
+/* Self-test of the bounded in-kernel waits (the pages have no counterpart; this checks
+ * the library's own failure reporting on a given device). Launches one cooperative
+ * kernel of one 32-thread block per SM whose blocks meet at a grid barrier of the same
+ * kind the layer kernels use. Block `withhold` (0 <= withhold < SM count) never arrives;
+ * withhold < 0 lets every block arrive. Waiting blocks give up after limit_ns
+ * (1 ns .. 1 s), record the timeout in the error word of `workspace` and return, so the
+ * device stays usable. workspace == NULL uses the allocation-free scratch of the current
+ * device. Afterwards redmoe_check_timeout reports REDMOE_ERR_TIMEOUT (withhold >= 0) or
+ * REDMOE_OK (withhold < 0, unless an earlier timeout is still recorded); clear it with
+ * redmoe_workspace_init. Returns REDMOE_ERR_INVALID_ARG for a limit or block index out of
+ * range, REDMOE_ERR_WORKSPACE for a misaligned or short workspace. */
+redmoe_status redmoe_selftest_wait_limit(void *workspace, size_t workspace_bytes, int32_t withhold,
+                                         uint64_t limit_ns, void *stream);
+
+/* Debugging aid (no counterpart on the pages): enqueue on `stream` one kernel that fills
+ * the shared memory of every SM with the 32-bit `pattern` (0x7fc00000 is a quiet NaN).
+ * The layer kernels launched next on that stream then start on that pattern instead of
+ * on whatever an earlier launch left, so a kernel that reads its shared memory before the
+ * data has arrived produces visibly wrong results on every call, not only on the first
+ * call of a process. Not needed for correct use. */
+redmoe_status redmoe_fill_shared_memory(uint32_t pattern, void *stream);
 
 #ifdef __cplusplus
 }

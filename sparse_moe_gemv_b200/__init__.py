@@ -5,8 +5,9 @@ torch provides device memory and streams. The binding never computes a result it
 and has no fallback: if the library is missing it raises.
 
 Names match the C entry points (redmoe_forward, redmoe_router, redmoe_route_build,
-redmoe_forward_stack, redmoe_workspace_bytes, redmoe_workspace_init,
-redmoe_check_timeout, redmoe_status_string, redmoe_abi_version).
+redmoe_forward_stack, redmoe_forward_noalloc, redmoe_workspace_bytes,
+redmoe_workspace_init, redmoe_check_timeout, redmoe_selftest_wait_limit,
+redmoe_fill_shared_memory, redmoe_status_string, redmoe_abi_version).
 """
 
 from __future__ import annotations
@@ -27,7 +28,8 @@ STATUS = {0: "REDMOE_OK", 1: "REDMOE_ERR_INVALID_ARG", 2: "REDMOE_ERR_UNSUPPORTE
 # entry points declared in include/redmoe.h
 SYMBOLS = ("redmoe_abi_version", "redmoe_status_string", "redmoe_workspace_bytes", "redmoe_workspace_init",
            "redmoe_forward", "redmoe_router", "redmoe_route_build", "redmoe_forward_stack",
-           "redmoe_check_timeout", "redmoe_forward_noalloc")
+           "redmoe_check_timeout", "redmoe_forward_noalloc", "redmoe_selftest_wait_limit",
+           "redmoe_fill_shared_memory")
 
 _lock = threading.Lock()
 _lib = None
@@ -86,6 +88,10 @@ def load():
         lib.redmoe_check_timeout.argtypes = [P, P]
         lib.redmoe_forward_noalloc.restype = i32
         lib.redmoe_forward_noalloc.argtypes = [P, P, i32, P, P, P, P]
+        lib.redmoe_selftest_wait_limit.restype = i32
+        lib.redmoe_selftest_wait_limit.argtypes = [P, sz, i32, C.c_uint64, P]
+        lib.redmoe_fill_shared_memory.restype = i32
+        lib.redmoe_fill_shared_memory.argtypes = [C.c_uint32, P]
         if lib.redmoe_abi_version() != ABI_VERSION:
             raise RuntimeError("libredmoe.so ABI version mismatch")
         _lib = lib
@@ -154,9 +160,10 @@ def redmoe_workspace_bytes(layer: Layer, T: int) -> int:
     return int(load().redmoe_workspace_bytes(layer.ref, int(T)))
 
 
-def redmoe_workspace_init(workspace: torch.Tensor, stream=None) -> None:
-    _check(load().redmoe_workspace_init(_ptr(workspace), workspace.numel() * workspace.element_size(),
-                                        _stream(stream)), "redmoe_workspace_init")
+def redmoe_workspace_init(workspace: Optional[torch.Tensor], stream=None) -> None:
+    """Zero a workspace's control block; None: the allocation-free scratch of this device."""
+    nbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(load().redmoe_workspace_init(_ptr(workspace), nbytes, _stream(stream)), "redmoe_workspace_init")
 
 
 def new_workspace(layer: Layer, T: int, device=None) -> torch.Tensor:
@@ -214,7 +221,9 @@ def redmoe_forward_stack(layers: Sequence[Layer], xs: Sequence[torch.Tensor], ou
     _check(st, "redmoe_forward_stack")
 
 
-def redmoe_check_timeout(workspace: torch.Tensor, stream=None) -> None:
+def redmoe_check_timeout(workspace: Optional[torch.Tensor], stream=None) -> None:
+    """Raise REDMOE_ERR_TIMEOUT if a bounded in-kernel wait gave up; None: the
+    allocation-free scratch of this device."""
     _check(load().redmoe_check_timeout(_ptr(workspace), _stream(stream)), "redmoe_check_timeout")
 
 
@@ -226,8 +235,26 @@ def redmoe_forward_noalloc(layer: Layer, x: torch.Tensor, out: torch.Tensor, top
     must not touch the allocator, a plug-in without a memory budget of its own): the
     scratch is a fixed 1 MiB array inside the library, shared by every call on the
     device. Calls must not overlap on the GPU; the first call on a device must not be
-    made inside a stream capture (it looks up the array's address).
+    made inside a stream capture (it looks up the array's address). A bounded wait that
+    gave up is reported by redmoe_check_timeout(None) and cleared by
+    redmoe_workspace_init(None).
     """
     st = load().redmoe_forward_noalloc(layer.ref, _ptr(x), int(x.shape[0]), _ptr(out), _ptr(topk_ids),
                                        _ptr(topk_w), _stream(stream))
     _check(st, "redmoe_forward_noalloc")
+
+
+def redmoe_selftest_wait_limit(workspace: Optional[torch.Tensor], withhold: int, limit_ns: int, stream=None) -> None:
+    """Run the bounded-wait self-test: block `withhold` skips a grid barrier, the others
+    give up after limit_ns and record a timeout (read it with redmoe_check_timeout)."""
+    nbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(load().redmoe_selftest_wait_limit(_ptr(workspace), nbytes, int(withhold), int(limit_ns), _stream(stream)),
+           "redmoe_selftest_wait_limit")
+
+
+NAN_PATTERN = 0x7FC00000
+
+
+def redmoe_fill_shared_memory(pattern: int = NAN_PATTERN, stream=None) -> None:
+    """Fill every SM's shared memory with a 32-bit pattern before the next launch."""
+    _check(load().redmoe_fill_shared_memory(int(pattern) & 0xFFFFFFFF, _stream(stream)), "redmoe_fill_shared_memory")

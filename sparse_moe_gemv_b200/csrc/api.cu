@@ -45,6 +45,43 @@ bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) %
 
 int elems_per_chunk(int dt) { return dt == DT_F32 ? 4 : (dt == DT_BF16 ? 8 : 32); }
 
+// Workspace carve-up of the router entry point and of the batched path.
+struct BatchWs {
+    size_t logits, sgate, total;
+};
+BatchWs batch_ws_layout(int T, int E) {
+    BatchWs b;
+    size_t o = 256;
+    b.logits = o; o = align256(o + 4ull * T * E);
+    b.sgate = o; o = align256(o + 4ull * T);
+    b.total = o;
+    return b;
+}
+
+size_t ws_bytes(const redmoe_layer* L, int T) {
+    size_t need = 256;
+    if (T <= DECODE_MAX_T) {
+        const DecodeWs d = decode_ws_layout(T, L->n_experts, L->top_k, L->inter, L->shared_inter);
+        need = d.total > need ? d.total : need;
+    } else if (batch_shape_ok(L)) {
+        const BatchLayout g = batch_layout(T, L->n_experts, L->top_k, L->hidden, L->inter);
+        need = g.total > need ? g.total : need;
+    }
+    const BatchWs b = batch_ws_layout(T, L->n_experts);
+    need = b.total > need ? b.total : need;
+    return need;
+}
+
+redmoe_status check_ws(const redmoe_layer* L, int T, const void* ws, size_t bytes) {
+    if (!ws || !aligned(ws, 256)) return REDMOE_ERR_WORKSPACE;
+    if (bytes < ws_bytes(L, T)) return REDMOE_ERR_WORKSPACE;
+    return REDMOE_OK;
+}
+
+redmoe_status cuda_ok(cudaError_t e) { return e == cudaSuccess ? REDMOE_OK : REDMOE_ERR_CUDA; }
+
+}  // namespace
+
 // Shape, dtype and pointer checks common to every layer entry point.
 redmoe_status check_layer(const redmoe_layer* L) {
     if (!L) return REDMOE_ERR_INVALID_ARG;
@@ -97,45 +134,6 @@ DecLayer dec_layer(const redmoe_layer* L, const void* x, float* out, int32_t* id
     return d;
 }
 
-// Workspace carve-up of the router entry point and of the batched path.
-struct BatchWs {
-    size_t logits, sgate, total;
-};
-BatchWs batch_ws_layout(int T, int E) {
-    BatchWs b;
-    size_t o = 256;
-    b.logits = o; o = align256(o + 4ull * T * E);
-    b.sgate = o; o = align256(o + 4ull * T);
-    b.total = o;
-    return b;
-}
-
-size_t ws_bytes(const redmoe_layer* L, int T) {
-    size_t need = 256;
-    if (T <= DECODE_MAX_T) {
-        const DecodeWs d = decode_ws_layout(T, L->n_experts, L->top_k, L->inter, L->shared_inter);
-        need = d.total > need ? d.total : need;
-    } else if (batch_shape_ok(L)) {
-        const BatchLayout g = batch_layout(T, L->n_experts, L->top_k, L->hidden, L->inter);
-        need = g.total > need ? g.total : need;
-    }
-    const BatchWs b = batch_ws_layout(T, L->n_experts);
-    need = b.total > need ? b.total : need;
-    return need;
-}
-
-redmoe_status check_ws(const redmoe_layer* L, int T, const void* ws, size_t bytes) {
-    if (!ws || !aligned(ws, 256)) return REDMOE_ERR_WORKSPACE;
-    if (bytes < ws_bytes(L, T)) return REDMOE_ERR_WORKSPACE;
-    return REDMOE_OK;
-}
-
-redmoe_status cuda_ok(cudaError_t e) { return e == cudaSuccess ? REDMOE_OK : REDMOE_ERR_CUDA; }
-
-}  // namespace
-
-// Layer validation for redmoe_forward_noalloc (same rules as the other entry points).
-redmoe_status check_layer_for_noalloc(const redmoe_layer* L) { return check_layer(L); }
 
 }  // namespace redmoe
 
@@ -163,7 +161,12 @@ size_t redmoe_workspace_bytes(const redmoe_layer* L, int32_t T) {
 }
 
 redmoe_status redmoe_workspace_init(void* workspace, size_t workspace_bytes, void* stream) {
-    if (!workspace || !aligned(workspace, 256) || workspace_bytes < 256) return REDMOE_ERR_WORKSPACE;
+    if (!workspace) {  // the allocation-free scratch of this device
+        void* scratch = noalloc_scratch_address();
+        if (!scratch) return REDMOE_ERR_CUDA;
+        return cuda_ok(cudaMemsetAsync(scratch, 0, 256, static_cast<cudaStream_t>(stream)));
+    }
+    if (!aligned(workspace, 256) || workspace_bytes < 256) return REDMOE_ERR_WORKSPACE;
     return cuda_ok(cudaMemsetAsync(workspace, 0, 256, static_cast<cudaStream_t>(stream)));
 }
 
@@ -261,7 +264,11 @@ redmoe_status redmoe_forward_stack(const redmoe_layer* layers, int32_t n_layers,
 }
 
 redmoe_status redmoe_check_timeout(const void* workspace, void* stream) {
-    if (!workspace || !aligned(workspace, 256)) return REDMOE_ERR_WORKSPACE;
+    if (!workspace) {  // the allocation-free scratch of this device
+        workspace = noalloc_scratch_address();
+        if (!workspace) return REDMOE_ERR_CUDA;
+    }
+    if (!aligned(workspace, 256)) return REDMOE_ERR_WORKSPACE;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (cudaStreamSynchronize(s) != cudaSuccess) return REDMOE_ERR_CUDA;
     Control c;

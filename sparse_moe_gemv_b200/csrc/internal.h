@@ -41,6 +41,16 @@ struct DecLayer {
     float* w;
 };
 
+// The decode kernel's view of one redmoe_layer called on (x, out, ids, w).
+DecLayer dec_layer(const redmoe_layer* L, const void* x, float* out, int32_t* ids, float* w);
+
+// Layer validation shared by every entry point (shape, dtype combination, pointers).
+redmoe_status check_layer(const redmoe_layer* L);
+
+// Device address of the allocation-free scratch array on the current device (looked up
+// once per device); NULL on a CUDA error.
+void* noalloc_scratch_address();
+
 // Workspace carve-up of the decode path (byte offsets from the workspace base).
 struct DecodeWs {
     size_t logits, sgate, hsh, hrt, total;

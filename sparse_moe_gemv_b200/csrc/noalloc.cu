@@ -16,9 +16,14 @@
 // cudaGetSymbolAddress while that device is current and caches it; make that first call
 // outside any stream capture. Every call on a device shares the one array: calls that
 // may overlap on the GPU (different streams without ordering) race on it and must not
-// be issued. Each call clears the array's 256-byte control block with an asynchronous
-// memset (no allocation) before the kernel, because the kernel's grid barrier expects it
-// at zero.
+// be issued.
+//
+// The array starts with the same 256-byte control block as a workspace. Before each
+// launch a call clears the two grid-barrier counters (an asynchronous 8-byte memset, no
+// allocation), so that a launch that failed part-way cannot leave them dirty. It does
+// not clear the error word: a bounded in-kernel wait that gave up stays recorded until
+// the caller reads it with redmoe_check_timeout(NULL, stream) and clears it with
+// redmoe_workspace_init(NULL, 0, stream).
 #include <mutex>
 
 #include "common.cuh"
@@ -34,8 +39,10 @@ static __device__ __align__(256) unsigned char g_noalloc_scratch[NOALLOC_SCRATCH
 
 constexpr int MAX_DEVICES = 64;
 
+}  // namespace
+
 // Device address of g_noalloc_scratch on the current device, looked up once per device.
-void* scratch_address() {
+void* noalloc_scratch_address() {
     static std::mutex mu;
     static void* addr[MAX_DEVICES] = {};
     int dev = 0;
@@ -49,17 +56,13 @@ void* scratch_address() {
     return addr[dev];
 }
 
-}  // namespace
-
-redmoe_status check_layer_for_noalloc(const redmoe_layer* L);
-
 }  // namespace redmoe
 
 using namespace redmoe;
 
 extern "C" redmoe_status redmoe_forward_noalloc(const redmoe_layer* L, const void* x, int32_t T, float* out,
                                                 int32_t* topk_ids, float* topk_w, void* stream) {
-    redmoe_status st = check_layer_for_noalloc(L);
+    redmoe_status st = check_layer(L);
     if (st != REDMOE_OK) return st;
     if (T < 0) return REDMOE_ERR_INVALID_ARG;
     if (T == 0) return REDMOE_OK;
@@ -70,29 +73,11 @@ extern "C" redmoe_status redmoe_forward_noalloc(const redmoe_layer* L, const voi
     if (T > DECODE_MAX_T) return REDMOE_ERR_UNSUPPORTED;
     const DecodeWs need = decode_ws_layout(T, L->n_experts, L->top_k, L->inter, L->shared_inter);
     if (need.total > NOALLOC_SCRATCH_BYTES) return REDMOE_ERR_WORKSPACE;
-    void* ws = scratch_address();
+    void* ws = noalloc_scratch_address();
     if (!ws) return REDMOE_ERR_CUDA;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    if (cudaMemsetAsync(ws, 0, 256, s) != cudaSuccess) return REDMOE_ERR_CUDA;
-    DecLayer d;
-    d.router_w = L->router_w;
-    d.router_bias = L->router_bias;
-    d.shared_gate_w = L->shared_gate_w;
-    d.w_gate = L->w_gate;
-    d.w_up = L->w_up;
-    d.w_down = L->w_down;
-    d.s_gate = static_cast<const uint16_t*>(L->s_gate);
-    d.s_up = static_cast<const uint16_t*>(L->s_up);
-    d.s_down = static_cast<const uint16_t*>(L->s_down);
-    d.sh_gate = L->sh_gate;
-    d.sh_up = L->sh_up;
-    d.sh_down = L->sh_down;
-    d.sh_s_gate = static_cast<const uint16_t*>(L->sh_s_gate);
-    d.sh_s_up = static_cast<const uint16_t*>(L->sh_s_up);
-    d.sh_s_down = static_cast<const uint16_t*>(L->sh_s_down);
-    d.x = x;
-    d.out = out;
-    d.ids = topk_ids;
-    d.w = topk_w;
+    static_assert(offsetof(Control, err) == 8, "the barrier counters are the first 8 bytes");
+    if (cudaMemsetAsync(ws, 0, offsetof(Control, err), s) != cudaSuccess) return REDMOE_ERR_CUDA;
+    const DecLayer d = dec_layer(L, x, out, topk_ids, topk_w);
     return launch_decode(L, &d, 1, T, ws, s, nullptr);
 }

@@ -133,8 +133,29 @@ def test_router_and_stack_reject_bad_arguments(lib):
                                     C.cast(ptrs, C.c_void_p), C.cast(ptrs, C.c_void_p),
                                     C.cast(ptrs, C.c_void_p), FAKE, 1 << 30, 0) == INVALID
     assert lib.redmoe_forward_stack(None, 2, None, 1, None, None, None, FAKE, 1 << 30, 0) == INVALID
-    assert lib.redmoe_workspace_init(None, 256, 0) == WORKSPACE
-    assert lib.redmoe_check_timeout(None, 0) == WORKSPACE
+    # a misaligned workspace is refused before any CUDA call
+    assert lib.redmoe_workspace_init(C.c_void_p(FAKE + 16), 256, 0) == WORKSPACE
+    assert lib.redmoe_workspace_init(FAKE, 255, 0) == WORKSPACE
+    assert lib.redmoe_check_timeout(C.c_void_p(FAKE + 16), 0) == WORKSPACE
+
+
+def test_null_workspace_means_the_noalloc_scratch(lib):
+    """NULL selects the library's own scratch array; with no CUDA device the lookup of
+    its address fails, which is a CUDA error, not a workspace error."""
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("needs a host without a CUDA device")
+    CUDA = 4
+    assert lib.redmoe_workspace_init(None, 0, 0) == CUDA
+    assert lib.redmoe_check_timeout(None, 0) == CUDA
+
+
+def test_selftest_rejects_bad_limits_before_touching_cuda(lib):
+    f = lib.redmoe_selftest_wait_limit
+    assert f(FAKE, 256, 0, 0, 0) == INVALID
+    assert f(FAKE, 256, 0, 2_000_000_000, 0) == INVALID
+    assert f(C.c_void_p(FAKE + 16), 256, 0, 1000, 0) == WORKSPACE
+    assert f(FAKE, 128, 0, 1000, 0) == WORKSPACE
 
 
 def test_noalloc_rejects_before_touching_cuda(lib):

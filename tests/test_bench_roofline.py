@@ -72,9 +72,11 @@ def test_workload_table(bench):
 def test_traffic_figure_needs_matching_sources(bench, tmp_path, monkeypatch):
     with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
         committed = json.load(f)
-    # the committed figures name the current sources, so they are reported
+    # a committed figure is reported exactly when it names the current sources
     for wl, d in committed.items():
-        assert bench.profile_traffic(wl) == d["dram_bytes_per_launch"], wl
+        files = bench.PREFILL_SOURCES if wl.startswith("prefill") else bench.DECODE_SOURCES
+        current = d["source_digest"] == bench.source_digest(files)
+        assert bench.profile_traffic(wl) == (d["dram_bytes_per_launch"] if current else None), wl
     # a workload without a capture reports none
     assert bench.profile_traffic("prefill_uniform") is None
     # a figure taken on other sources is not reported

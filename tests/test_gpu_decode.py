@@ -128,3 +128,29 @@ def test_router_entry_point(gpu_lib):
             sets, ex = candidate_sets(r["logits"][t], shape.k)
             assert tuple(sorted(ids[t].tolist())) in sets
             assert check_order(r["logits"][t], ids[t].cpu().numpy())
+
+
+@pytest.mark.parametrize("name,T", [("bf16", 1), ("bf16", 2), ("bf16", 3), ("bf16", 4), ("int4", 1), ("int4", 3),
+                                    ("tiny", 4)])
+def test_decode_after_shared_memory_poison(gpu_lib, name, T):
+    """Every SM's shared memory is filled with NaN right before the call, so a read of a
+    ring stage, of x or of h ahead of its data shows up in the results of this call."""
+    shape = {"bf16": QWEN, "int4": QWEN_INT4, "tiny": TINY}[name]
+    if name == "tiny":
+        L = {k: (v.cuda() if v is not None else None) for k, v in mi.make_layer(shape, 5, "cpu").items()}
+        x = mi.make_x(shape, T, 5, "cpu").cuda()
+    else:
+        L = _dev_layer(shape, 5000 + T)
+        x = mi.make_x(shape, T, 5000 + T, "cuda")
+    lay = smg.Layer.from_shape(L, shape)
+    ws = smg.new_workspace(lay, T)
+    ot, wt = tolerances(shape)
+    for call in range(2):
+        out = torch.full((T, shape.H), float("nan"), device="cuda")
+        ids = torch.full((T, shape.k), -1, dtype=torch.int32, device="cuda")
+        w = torch.full((T, shape.k), float("nan"), device="cuda")
+        smg.redmoe_fill_shared_memory()
+        smg.redmoe_forward(lay, x, out, ids, w, ws)
+        smg.redmoe_check_timeout(ws)
+        assert bool(torch.isfinite(out).all()), f"{name} T={T} call {call}: non-finite outputs"
+        assert_layer_parity(shape, L, x, out, ids, w, ot, wt, f"poisoned {name} T={T} call {call}")

@@ -49,33 +49,37 @@ def test_qwen_layer_batched(gpu_lib, T):
     shape = QWEN
     L = mi.make_layer(shape, 3100 + T, "cuda")
     x = mi.make_x(shape, T, 3100 + T, "cuda")
-    out, ids, w, _ = _run(shape, L, x)
+    out, ids, w, dbg = _run(shape, L, x, dbg=True)
     ot, wt = tolerances(shape)
     assert_layer_parity(shape, L, x, out, ids, w, ot, wt, f"qwen batched T={T}")
+    _assert_grouping_of_gpu_ids(ids, dbg, shape.E)
 
 
 def test_prefill_chunk_zipf_2048(gpu_lib):
-    """The 2048-token prefill chunk with Zipf(1.1) router offsets: every token's ids and
-    weights, the grouping (counts and offsets exact; the permutation exact when no token
-    sits on a near-tie), and the outputs of a sample of 256 tokens."""
+    """The 2048-token prefill chunk with Zipf(1.1) router offsets: every token's ids,
+    weights and output row (tolerance relative to the RMS of the whole [T, H] output),
+    and the grouping, bit-exact against the oracle's stable grouping of the GPU's own ids
+    (the reference for a near-tie token is then still unique)."""
     shape = QWEN_ZIPF
     T = 2048
     L = mi.make_layer(shape, 3000, "cuda")
     x = mi.make_x(shape, T, 3000, "cuda")
     out, ids, w, dbg = _run(shape, L, x, dbg=True)
-    rows = np.sort(np.random.default_rng(0).choice(T, 256, replace=False))
     ot, wt = tolerances(shape)
-    r = assert_layer_parity(shape, L, x, out, ids, w, ot, wt, "prefill zipf", rows=rows)
-    ref = r["ref"]
-    c_ref, o_ref, p_ref = oracle.route_build(ref["ids"], shape.E)
-    np.testing.assert_array_equal(dbg[0].cpu().numpy(), c_ref)
-    np.testing.assert_array_equal(dbg[1].cpu().numpy(), o_ref)
-    perm = dbg[2].cpu().numpy()
-    if not ref["exempt"].any():
-        np.testing.assert_array_equal(perm, p_ref)
-    assert sorted(perm.tolist()) == list(range(T * shape.k))
+    r = assert_layer_parity(shape, L, x, out, ids, w, ot, wt, "prefill zipf")
+    _assert_grouping_of_gpu_ids(ids, dbg, shape.E)
+    c_ref = oracle.route_build(r["ref"]["ids"], shape.E)[0]
     # the workload's shape: a few hot experts take hundreds of tokens, most take none
     assert int((c_ref >= 100).sum()) >= 5 and int((c_ref == 0).sum()) >= 200
+
+
+def _assert_grouping_of_gpu_ids(ids, dbg, E):
+    """counts, offsets and perm of the forward equal the oracle's grouping of the ids the
+    GPU chose, bit for bit."""
+    c_ref, o_ref, p_ref = oracle.route_build(ids.cpu().numpy(), E)
+    np.testing.assert_array_equal(dbg[0].cpu().numpy(), c_ref)
+    np.testing.assert_array_equal(dbg[1].cpu().numpy(), o_ref)
+    np.testing.assert_array_equal(dbg[2].cpu().numpy(), p_ref)
 
 
 MID = mi.LayerShape(H=512, E=40, k=3, I=256, Is=256, sigma=0.04)
@@ -106,20 +110,17 @@ def test_top1_routing_batched(gpu_lib):
 
 def test_chunk_4096_all_experts(gpu_lib):
     """A 4096-token chunk with unbiased routing: every expert receives tokens and every CTA
-    of the grouped GEMMs runs many tiles. Ids and weights of every token, the grouping,
-    and the outputs of a sample of 64 tokens."""
+    of the grouped GEMMs runs many tiles. Ids, weights and output rows of every token,
+    and the grouping bit-exact against the oracle's grouping of the GPU's ids."""
     shape = QWEN
     T = 4096
     L = mi.make_layer(shape, 4096, "cuda")
     x = mi.make_x(shape, T, 4096, "cuda")
     out, ids, w, dbg = _run(shape, L, x, dbg=True)
-    rows = np.sort(np.random.default_rng(1).choice(T, 64, replace=False))
     ot, wt = tolerances(shape)
-    r = assert_layer_parity(shape, L, x, out, ids, w, ot, wt, "chunk 4096", rows=rows)
-    c_ref, o_ref, p_ref = oracle.route_build(r["ref"]["ids"], shape.E)
-    np.testing.assert_array_equal(dbg[0].cpu().numpy(), c_ref)
-    np.testing.assert_array_equal(dbg[1].cpu().numpy(), o_ref)
-    assert int((c_ref > 0).sum()) == shape.E
+    assert_layer_parity(shape, L, x, out, ids, w, ot, wt, "chunk 4096")
+    _assert_grouping_of_gpu_ids(ids, dbg, shape.E)
+    assert int((dbg[0] > 0).sum()) == shape.E
 
 
 def test_batched_repeat_is_stable(gpu_lib):

@@ -1,15 +1,16 @@
 """redmoe_forward_noalloc: the decode-size forward for callers that cannot allocate
 device memory (strict stream capture, allocator-free hot loops, plug-ins without a
 memory budget). Its scratch is a fixed array inside the library; the test checks,
-through the C ABI, that two calls in a row give the same result as redmoe_forward with
-a caller workspace. The file name makes pytest collect it last."""
+through the C ABI, that two calls in a row give the result of redmoe_forward with a
+caller workspace and of the fp64 oracle, and that the scratch's error word reads clean.
+The file name makes pytest collect it last."""
 
 import pytest
 import torch
 
 import moe_inputs as mi
 import sparse_moe_gemv_b200 as smg
-from parity import tolerances
+from parity import assert_layer_parity, tolerances
 
 pytestmark = pytest.mark.gpu
 
@@ -35,8 +36,9 @@ def test_noalloc_matches_workspace_forward_twice(gpu_lib, T):
         ids = torch.full((T, shape.k), -1, dtype=torch.int32, device="cuda")
         w = torch.full((T, shape.k), float("nan"), device="cuda")
         smg.redmoe_forward_noalloc(lay, x, out, ids, w)
-        torch.cuda.synchronize()
+        smg.redmoe_check_timeout(None)
         assert torch.equal(ids, ref_ids), f"call {call}: ids differ"
         assert float((w - ref_w).abs().max()) <= w_tol, f"call {call}: weights differ"
         err = float((out.double() - ref.double()).abs().max())
         assert err <= out_tol * rms, f"call {call}: max err {err:.3e} > {out_tol} * RMS {rms:.3e}"
+        assert_layer_parity(shape, L, x, out, ids, w, out_tol, w_tol, f"noalloc T={T} call {call}")
