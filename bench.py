@@ -12,11 +12,15 @@ Workloads (synthetic seeded layers of the Qwen3-Next-80B-A3B MoE shape: hidden 2
   prefill     a 2048-token chunk through one bf16 layer with Zipf(1.1) router offsets
 
 One JSON line on rank 0: the device-timed throughput (CUDA events on the launching
-stream, graph replay of the steps, barrier + synchronize around the timed region, max
-over ranks), the roofline of the dominant kernel, the end-to-end figure through the C
-ABI with pinned host buffers, the fp64 oracle on the host cores, and the SM clocks seen
-during the timed region. The path does not shard (one layer fits one GPU): with N > 1
-every rank runs its own replica ("replicas only"), the value is the sum over ranks.
+stream, the timed steps replayed from CUDA graphs, barrier + synchronize around the
+timed region, max over ranks), the roofline of the dominant kernel, the end-to-end
+figure through the C ABI with pinned host buffers, the fp64 oracle on the host cores,
+and the SM clocks seen during the timed region. A step of a stack workload is one token
+(T rows) through the whole stack, so its tokens/s are model-depth tokens. The default
+run (decode_t1) adds one object per other workload (fewrow_t2, fewrow_t3, int4_48,
+prefill, prefill_uniform), each with its own roofline, end-to-end figure and clocks.
+The path does not shard (one layer fits one GPU): with N > 1 every rank runs its own
+replica ("replicas only"), the value is the sum over ranks.
 """
 
 from __future__ import annotations
@@ -125,7 +129,7 @@ def profile_traffic(workload):
     if not os.path.exists(p):
         return None
     d = json.load(open(p)).get(workload)
-    files = PREFILL_SOURCES if workload == "prefill" else DECODE_SOURCES
+    files = PREFILL_SOURCES if workload.startswith("prefill") else DECODE_SOURCES
     if not d or d.get("source_digest") != source_digest(files):
         return None
     return d.get("dram_bytes_per_launch")
@@ -232,6 +236,28 @@ def job_throughput(units, seconds, world):
 
 
 # ------------------------------------------------------------- CPU baseline
+def _used_experts(lay, shape, x):
+    """Experts the oracle's own routing of x selects (so that only those are fetched)."""
+    import oracle
+    r = oracle.router(lay, shape, x)
+    return sorted(set(r["ids"].reshape(-1).tolist()))
+
+
+def _host_layer(L, shape, x):
+    import oracle  # noqa: F401
+    lay = mi.layer_to_numpy(L, experts=[])
+    return mi.layer_to_numpy(L, experts=_used_experts(lay, shape, x))
+
+
+def _time_oracle(fn, threads):
+    import oracle
+    oracle.set_num_threads(threads)
+    fn()  # warm-up call (page-in, thread start)
+    t0 = time.perf_counter()
+    fn()
+    return time.perf_counter() - t0
+
+
 def cpu_oracle_sample(wl, seconds=10.0):
     """The fp64 oracle on the host cores over a bounded sample of the workload: decode
     tokens through layer 0 of the workload (one oracle call, OpenMP over tokens)."""
@@ -239,21 +265,55 @@ def cpu_oracle_sample(wl, seconds=10.0):
     shape = wl["shape"]
     cores = oracle.num_threads()
     L = mi.make_layer(shape, wl["seed"], "cuda")
+    x1 = mi.to_numpy(mi.make_x(shape, 1, wl["seed"] + 99, "cpu"))
     lay = mi.layer_to_numpy(L)
     del L
-    x1 = mi.to_numpy(mi.make_x(shape, 1, wl["seed"] + 99, "cpu"))
-    t0 = time.perf_counter()
-    oracle.forward(lay, shape, x1)
-    t1 = time.perf_counter() - t0
+    t1 = _time_oracle(lambda: oracle.forward(lay, shape, x1), cores)
     n = int(max(cores, min(4096, seconds * cores / max(t1, 1e-3))))
     n = max(cores, (n // cores) * cores)
     x = mi.to_numpy(mi.make_x(shape, n, wl["seed"] + 123, "cpu"))
     t0 = time.perf_counter()
     oracle.forward(lay, shape, x)
     el = time.perf_counter() - t0
+    # one thread on one decode token (the single-thread time of a T = 1 layer call)
+    t_single = _time_oracle(lambda: oracle.forward(lay, shape, x1), 1)
+    oracle.set_num_threads(cores)
     return {"value": n / el, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+            "omp_num_threads": cores, "omp_env": os.environ.get("OMP_NUM_THREADS"), "nproc": os.cpu_count(),
             "sample": f"{n} decode tokens through one {wl['desc']} layer, one oracle call "
-                      f"(fp64, OpenMP over tokens), {el:.1f} s wall"}
+                      f"(fp64, OpenMP over tokens), {el:.1f} s wall",
+            "single_thread": {"value": 1.0 / t_single, "unit": "tokens/s", "seconds_per_call": t_single,
+                              "sample": "one T=1 call of the same layer on one thread"}}
+
+
+def cpu_oracle_stack(wl, B, T=2):
+    """The oracle over the 12-layer few-row stack at T tokens (one step = T tokens through
+    all layers), every thread of the host; experts fetched as the oracle routes them."""
+    import oracle
+    shape = wl["shape"]
+    cores = oracle.num_threads()
+    hl = []
+    for l in range(len(B["tens"])):
+        x = mi.to_numpy(B["xs"][l][:T])
+        hl.append((_host_layer(B["tens"][l], shape, x), x))
+    el = _time_oracle(lambda: [oracle.forward(lay, shape, x) for lay, x in hl], cores)
+    return {"value": T / el, "unit": "tokens/s", "cores": min(cores, T), "threads": cores,
+            "seconds_per_step": el,
+            "sample": f"one step: T={T} tokens through {len(hl)} distinct layers, fp64 oracle "
+                      f"(threads beyond T idle: OpenMP over a call's tokens)"}
+
+
+def cpu_oracle_prefill(wl, B, n=256):
+    """The oracle on the first n tokens of the prefill chunk (a bounded sample)."""
+    import oracle
+    shape = wl["shape"]
+    cores = oracle.num_threads()
+    x = mi.to_numpy(B["xs"][0][:n])
+    lay = _host_layer(B["tens"][0], shape, x)
+    el = _time_oracle(lambda: oracle.forward(lay, shape, x), cores)
+    return {"value": n / el, "unit": "tokens/s", "cores": cores, "seconds": el,
+            "sample": f"the first {n} of the {wl['T']} tokens of the chunk, one oracle call "
+                      f"({len(lay['w_gate'])} experts fetched), fp64, OpenMP over tokens"}
 
 
 def reference_arm(args, wl, world, rank):
@@ -273,7 +333,7 @@ def reference_arm(args, wl, world, rank):
         del L
     torch.cuda.empty_cache()
     xs = [mi.to_numpy(mi.make_x(shape, T, wl["seed"] + 7 * s, "cpu")) for s in range(4)]
-    tokens_per_step = T * (wl["layers"] if wl["stack"] else 1)
+    tokens_per_step = T  # a stack step is T tokens through every layer
 
     def step(s):
         for l in range(wl["layers"] if wl["stack"] else 1):
@@ -308,9 +368,11 @@ def reference_arm(args, wl, world, rank):
 
 
 # ------------------------------------------------------------------ GPU arm
-def build_workload(wl, smg):
+def build_workload(wl, smg, tens=None):
+    """Device layers (or the given ones), inputs, outputs and a workspace for the workload."""
     shape, T, nl = wl["shape"], wl["T"], wl["layers"]
-    tens = [mi.make_layer(shape, wl["seed"] + l, "cuda") for l in range(nl)]
+    if tens is None:
+        tens = [mi.make_layer(shape, wl["seed"] + l, "cuda") for l in range(nl)]
     lays = [smg.Layer.from_shape(t, shape) for t in tens]
     xs = [mi.make_x(shape, T, wl["seed"] + l, "cuda") for l in range(nl)]
     outs = [torch.empty(T, shape.H, device="cuda") for _ in range(nl)]
@@ -342,31 +404,59 @@ def capture(step, n, stream):
     return g
 
 
-def gpu_arm(args, wl, world, rank, local):
+class GraphRunner:
+    """Replays n steps as whole CUDA graphs: full rotations of the layers, then one graph
+    of the remaining steps, so that no eager host call sits between timed launches."""
+
+    def __init__(self, step, chunk, stream):
+        self.step, self.chunk, self.stream = step, chunk, stream
+        self.graphs = {}
+
+    def _graph(self, n):
+        if n not in self.graphs:
+            self.graphs[n] = capture(self.step, n, self.stream)
+        return self.graphs[n]
+
+    def prepare(self, *counts):
+        for n in counts:
+            full, rem = divmod(n, self.chunk)
+            if full:
+                self._graph(self.chunk)
+            if rem:
+                self._graph(rem)
+
+    def run(self, n):
+        full, rem = divmod(n, self.chunk)
+        g = self.graphs.get(self.chunk)
+        for _ in range(full):
+            g.replay()
+        if rem:
+            self.graphs[rem].replay()
+
+
+def distinct_experts(B):
+    """Distinct routed experts of each layer's last call, from the ids it returned."""
+    return [len(set(ids.view(-1).tolist())) for ids in B["ids"]]
+
+
+def gpu_arm(args, wl, world, rank, local, B=None, name=None):
     import sparse_moe_gemv_b200 as smg
     smg.load()
     shape, T = wl["shape"], wl["T"]
-    B = build_workload(wl, smg)
+    if B is None:
+        B = build_workload(wl, smg)
     stream = torch.cuda.Stream()
     step, launches_per_step = make_step(wl, smg, B, stream)
     with torch.cuda.stream(stream):
         step(0)  # one eager call: per-device set-up (attributes, driver entry points) outside capture
     torch.cuda.synchronize()
-    # graphs: one rotation of the layers per replay (stack workloads: one stack per replay)
-    chunk = 1 if wl["stack"] else wl["layers"]
-    graph = capture(step, chunk, stream)
     K, W = args.steps, args.warmup
+    runner = GraphRunner(step, 1 if wl["stack"] else wl["layers"], stream)
+    runner.prepare(W, K)
     torch.cuda.synchronize()
 
-    def run(nsteps):
-        full, rem = divmod(nsteps, chunk)
-        for _ in range(full):
-            graph.replay()
-        for i in range(rem):
-            step(i)
-
     with torch.cuda.stream(stream):
-        run(W)
+        runner.run(W)
     torch.cuda.synchronize()
     smg.redmoe_check_timeout(B["work"], stream=stream)
 
@@ -377,21 +467,17 @@ def gpu_arm(args, wl, world, rank, local):
     with ClockSampler(local) as clk:
         with torch.cuda.stream(stream):
             ev0.record(stream)
-            run(K)
+            runner.run(K)
             ev1.record(stream)
         torch.cuda.synchronize()
     barrier(world)
     smg.redmoe_check_timeout(B["work"], stream=stream)
     el_ms = ev0.elapsed_time(ev1)
-    tokens_per_step = T * (wl["layers"] if wl["stack"] else 1)
+    tokens_per_step = T  # one layer call, or T tokens through the whole stack
     value = job_throughput(K * tokens_per_step, el_ms / 1e3, world)  # this rank's time in
     el_ms = max_over_ranks(el_ms, world)
 
-    # distinct experts per layer call, from the ids of the last step of each layer
-    distinct = []
-    for l in range(wl["layers"]):
-        distinct.append(len(set(B["ids"][l].view(-1).tolist())))
-    layers_per_step = wl["layers"] if wl["stack"] else 1
+    distinct = distinct_experts(B)
     if wl["stack"]:
         bytes_per_launch = sum(layer_call_bytes(shape, T, d) for d in distinct)
     else:
@@ -400,18 +486,23 @@ def gpu_arm(args, wl, world, rank, local):
     launch_s = el_ms / 1e3 / launches
     hbm, bf16, bf16_sus, src = peaks()
     achieved = bytes_per_launch / launch_s / 1e9
+    key = name or args.workload
     if T > 4:
         # batched path: four kernels per step; the roofline is the tensor-core one of the layer
         flops = layer_flops(shape, T)
         step_s = el_ms / 1e3 / K
         tfl = flops / step_s / 1e12
         roof = {"bound": "tensor", "achieved": tfl, "peak": bf16, "unit": "TFLOP/s", "frac": tfl / bf16,
-                "traffic": profile_traffic(args.workload), "kernel": wl["kernel"], "flops_per_step": flops,
+                "traffic": profile_traffic(key), "kernel": wl["kernel"], "flops_per_step": flops,
                 "weight_bytes_per_step": bytes_per_launch, "hbm_gbs_of_weights": bytes_per_launch / step_s / 1e9,
+                "hbm_frac_of_weights": bytes_per_launch / step_s / 1e9 / hbm,
                 "peak_source": f"{src} (MEASURED_PEAKS.json bf16_tflops, burst)"}
         launches = K * 4
     else:
-        roof = None
+        roof = {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
+                "traffic": profile_traffic(key), "kernel": wl["kernel"], "bytes_per_launch": bytes_per_launch,
+                "launch_us": launch_s * 1e6, "distinct_experts_per_layer": statistics.mean(distinct),
+                "peak_source": f"{src} (MEASURED_PEAKS.json hbm_gbs)" if src == "measured" else "fallback"}
 
     # end to end through the C ABI with pinned host buffers: per step H2D x, forward, D2H out/ids/w
     e2e = e2e_arm(args, wl, smg, B, stream, world)
@@ -420,20 +511,19 @@ def gpu_arm(args, wl, world, rank, local):
         "ms_per_step": el_ms / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "bf16" if shape.expert_dtype == "bf16" else ("int4g32" if shape.expert_dtype == "int4g32" else "f32"),
         "data": "synthetic",
-        "config": {"workload": wl["desc"], "tokens_per_step": tokens_per_step, "layers_in_rotation": wl["layers"],
+        "config": {"workload": wl["desc"], "tokens_per_step": tokens_per_step, "layers": wl["layers"],
+                   "layers_per_step": wl["layers"] if wl["stack"] else 1,
                    "l2": "inputs larger than L2: each step reads a different layer's weights "
                          f"({wl['layers']} distinct layers)" if not wl["stack"] else
                          f"inputs larger than L2: {wl['layers']} distinct layers per step",
-                   "parallelism": "replicas" if world > 1 else "single GPU", "timing": "CUDA graph replay"},
-        "roofline": roof or {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
-                             "traffic": profile_traffic(args.workload), "kernel": wl["kernel"],
-                             "bytes_per_launch": bytes_per_launch, "launch_us": launch_s * 1e6,
-                             "peak_source": f"{src} (MEASURED_PEAKS.json hbm_gbs)" if src == "measured" else "fallback"},
+                   "parallelism": "replicas" if world > 1 else "single GPU",
+                   "timing": "CUDA graph replay of exactly the timed steps"},
+        "roofline": roof,
         "e2e": e2e,
         "gpu_launches": launches,
         "clocks": clk.summary(),
     }
-    return result
+    return result, B
 
 
 def e2e_arm(args, wl, smg, B, stream, world):
@@ -478,13 +568,32 @@ def e2e_arm(args, wl, smg, B, stream, world):
     stream.synchronize()
     el = time.perf_counter() - t0
     per = (nl if wl["stack"] else 1)
-    rate = job_throughput(n_e2e * T * per, el, world)  # this rank's wall time in
+    rate = job_throughput(n_e2e * T, el, world)  # this rank's wall time in; T tokens per step
     h2d = T * shape.H * xb * per
     d2h = (T * shape.H * 4 + T * shape.k * 8) * per
     return {"value": rate, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
             "d2h_bytes_per_step": d2h, "steps": n_e2e,
             "how": "redmoe_forward through the C ABI per step; pinned host x copied in, out/ids/w copied out, "
                    "host wall clock around the K steps"}
+
+
+SUB_WORKLOADS = ("fewrow_t2", "fewrow_t3", "int4_48", "prefill", "prefill_uniform")
+SUB_STEPS = {"fewrow_t2": 200, "fewrow_t3": 200, "int4_48": 100, "prefill": 50, "prefill_uniform": 30}
+
+
+def sub_result(res):
+    keep = ("value", "unit", "ms_per_step", "steps", "warmup", "dtype", "roofline", "e2e", "gpu_launches", "clocks")
+    d = {k: res[k] for k in keep}
+    d["workload"] = res["config"]["workload"]
+    d["tokens_per_step"] = res["config"]["tokens_per_step"]
+    return d
+
+
+def free(B):
+    if B is not None:
+        B.clear()
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
 
 
 def main():
@@ -495,7 +604,8 @@ def main():
     ap.add_argument("--workload", default="decode_t1", choices=sorted(WORKLOADS))
     ap.add_argument("--impl", default="redmoe", choices=["redmoe", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--no-prefill", action="store_true", help="skip the prefill summary of the default run")
+    ap.add_argument("--no-extra", action="store_true",
+                    help="default run: skip the objects of the other workloads")
     ap.add_argument("--layers", type=int, default=None,
                     help="override the number of distinct layers (small cases for profiler captures)")
     args = ap.parse_args()
@@ -512,17 +622,37 @@ def main():
         if world > 1:
             torch.distributed.destroy_process_group()
         return
-    res = gpu_arm(args, wl, world, rank, local)
-    if args.workload == "decode_t1" and not args.no_prefill:
-        torch.cuda.empty_cache()
-        pargs = argparse.Namespace(**{**vars(args), "steps": min(args.steps, 30), "warmup": 3, "workload": "prefill"})
-        pre = gpu_arm(pargs, WORKLOADS["prefill"], world, rank, local)
-        res["prefill"] = {"workload": WORKLOADS["prefill"]["desc"], "value": pre["value"], "unit": "tokens/s",
-                          "ms_per_step": pre["ms_per_step"], "steps": pre["steps"], "roofline": pre["roofline"],
-                          "e2e": pre["e2e"], "gpu_launches": pre["gpu_launches"], "clocks": pre["clocks"]}
+    cpu = world == 1 and rank == 0 and not args.no_cpu_baseline
+    res, B = gpu_arm(args, wl, world, rank, local)
+    free(B)
+    extra_cpu = {}
+    if args.workload == "decode_t1" and not args.no_extra:
+        fewrow_B = None
+        for name in SUB_WORKLOADS:
+            swl = WORKLOADS[name]
+            sargs = argparse.Namespace(**{**vars(args), "steps": min(args.steps, SUB_STEPS[name]), "warmup": 3,
+                                          "workload": name})
+            reuse = None
+            if name == "fewrow_t3" and fewrow_B is not None:
+                import sparse_moe_gemv_b200 as smg
+                reuse = build_workload(swl, smg, tens=fewrow_B["tens"])  # same 12 layers, T=3 buffers
+                free(fewrow_B)
+            sub, Bs = gpu_arm(sargs, swl, world, rank, local, B=reuse, name=name)
+            res[name] = sub_result(sub)
+            if cpu and name == "fewrow_t2":
+                extra_cpu["fewrow_t2_stack"] = cpu_oracle_stack(swl, Bs, T=2)
+            if cpu and name == "prefill":
+                extra_cpu["prefill_chunk"] = cpu_oracle_prefill(swl, Bs)
+            if name == "fewrow_t2":
+                fewrow_B = Bs  # the T=3 stack runs on the same 12 layers
+            else:
+                free(Bs)
+                if name == "fewrow_t3":
+                    fewrow_B = None
     if rank == 0:
-        if world == 1 and not args.no_cpu_baseline:
+        if cpu:
             res["cpu_baseline"] = cpu_oracle_sample(wl)
+            res["cpu_baseline"].update(extra_cpu)
         print(json.dumps(res), flush=True)
     if world > 1:
         torch.distributed.barrier()

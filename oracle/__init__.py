@@ -69,7 +69,10 @@ def _lib():
             lib.orc_route_build.argtypes = [i32, i32, i32, P, P, P, P]
             lib.orc_dequant_int4.argtypes = [i32, i32, P, P, P]
             lib.orc_renorm.argtypes = [i32, i32, P, P, P]
+            lib.orc_cache_route.argtypes = [i32, i32, i32, P, P, C.c_double, P, P, P]
             lib.orc_num_threads.argtypes = []
+            lib.orc_set_num_threads.argtypes = [i32]
+            lib.orc_set_num_threads.restype = None
             _handle = lib
     return _handle
 
@@ -214,6 +217,21 @@ def renorm(logits_row, ids):
     return w
 
 
+def cache_route(logits, cached, lam, k):
+    """Opt-in cache-aware routing of logits [T, E]: selection by z + lam * (max z - min z)
+    * cached, weights from the unbiased softmax renormalised over the selection.
+    Returns dict(ids [T,k] int32, w [T,k], biased [T,E])."""
+    logits = np.ascontiguousarray(logits, np.float64)
+    T, E = logits.shape
+    cached = np.ascontiguousarray(cached, np.uint8)
+    ids = np.zeros((T, k), np.int32)
+    w = np.zeros((T, k), np.float64)
+    biased = np.zeros((T, E), np.float64)
+    _check(_lib().orc_cache_route(T, E, k, _ptr(logits), _ptr(cached), float(lam), _ptr(ids), _ptr(w),
+                                  _ptr(biased)))
+    return dict(ids=ids, w=w, biased=biased)
+
+
 def route_build(ids, E):
     """Stable token->expert grouping: (counts [E], offsets [E+1], perm [T*k]) int32."""
     ids = np.ascontiguousarray(ids, np.int32)
@@ -237,3 +255,8 @@ def dequant_int4(packed, scales):
 
 def num_threads():
     return int(_lib().orc_num_threads())
+
+
+def set_num_threads(n):
+    """OpenMP threads of later oracle calls (timing only; results do not depend on it)."""
+    _lib().orc_set_num_threads(int(n))

@@ -137,6 +137,17 @@ int orc_num_threads(void)
 #endif
 }
 
+/* Threads of later calls (timing only: results do not depend on it). */
+void orc_set_num_threads(int32_t n)
+{
+#ifdef _OPENMP
+    if (n > 0)
+        omp_set_num_threads(n);
+#else
+    (void)n;
+#endif
+}
+
 /* ------------------------------------------------------------ int4 group-32 */
 int orc_dequant_int4(int32_t N, int32_t K, const uint8_t *packed, const uint16_t *scales, double *out)
 {
@@ -530,5 +541,64 @@ int orc_route_build(int32_t T, int32_t k, int32_t E, const int32_t *ids,
     for (long i = 0; i < (long)T * k; ++i)
         perm[cursor[ids[i]]++] = (int32_t)i;
     free(cursor);
+    return ORC_OK;
+}
+
+/* ------------------------------------------------- cache-aware routing (opt-in) */
+/* Routing with a bias towards experts the caller holds in a cache ("Research notes,
+ * October 2026", section 4, row "Cache-aware routing bias": z + lambda * Delta * cached,
+ * opt-in only because it changes outputs). The pages give only that expression; this
+ * oracle takes its plainest reading:
+ *   z[e]       the token's router logits (offset included), as from orc_router;
+ *   cached[e]  1 if expert e is resident in the caller's cache, else 0;
+ *   Delta      the token's logit range, max_e z[e] - min_e z[e], so that lambda is
+ *              dimensionless (lambda = 1 lets a cached expert at the lowest logit tie
+ *              the best uncached one);
+ *   selection  the k largest z[e] + lambda * Delta * cached[e], ties to the lower id;
+ *   weights    the softmax of the unbiased z over all E restricted to the selection and
+ *              renormalised: the bias changes which experts run, not how the selected
+ *              experts' outputs are mixed.
+ * lambda = 0 is plain routing. `biased` (T x E, may be NULL) receives the biased
+ * logits the selection ranks. */
+int orc_cache_route(int32_t T, int32_t E, int32_t k, const double *logits, const uint8_t *cached,
+                    double lambda, int32_t *ids, double *w, double *biased)
+{
+    if (T < 0 || E <= 0 || k <= 0 || k > E || lambda < 0.0 || (T > 0 && (!logits || !cached || !ids || !w)))
+        return ORC_ERR_ARG;
+    double *zb = malloc(sizeof(double) * (size_t)E);
+    unsigned char *taken = malloc((size_t)E);
+    if (!zb || !taken) {
+        free(zb);
+        free(taken);
+        return ORC_ERR_NOMEM;
+    }
+    for (long t = 0; t < T; ++t) {
+        const double *z = logits + t * E;
+        double zmax = z[0], zmin = z[0];
+        for (int e = 1; e < E; ++e) {
+            if (z[e] > zmax)
+                zmax = z[e];
+            if (z[e] < zmin)
+                zmin = z[e];
+        }
+        const double delta = zmax - zmin;
+        for (int e = 0; e < E; ++e)
+            zb[e] = z[e] + lambda * delta * (cached[e] ? 1.0 : 0.0);
+        if (biased)
+            memcpy(biased + t * E, zb, sizeof(double) * (size_t)E);
+        int32_t *id = ids + t * k;
+        topk_select(zb, E, k, id, taken);
+        /* softmax over all E of the unbiased logits, then the selection renormalised */
+        double zsum = 0.0;
+        for (int e = 0; e < E; ++e)
+            zsum += exp(z[e] - zmax);
+        double ps = 0.0;
+        for (int j = 0; j < k; ++j)
+            ps += exp(z[id[j]] - zmax) / zsum;
+        for (int j = 0; j < k; ++j)
+            w[t * k + j] = (exp(z[id[j]] - zmax) / zsum) / ps;
+    }
+    free(zb);
+    free(taken);
     return ORC_OK;
 }

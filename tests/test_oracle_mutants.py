@@ -1,7 +1,8 @@
 """The oracle's pins must catch plausible mistakes.
 
 Each case plants one mistake in a copy of moe_oracle.c (on the CPU), builds it, and
-runs the pin suite against that build in a child process: the suite has to fail.
+runs the pin suites (test_oracle_pins.py, test_oracle_cache_route.py) against that build
+in a child process: the suites have to fail.
 """
 
 import os
@@ -31,6 +32,11 @@ MUTANTS = {
                                 "w[j] = (exp(logits_row[ids[j]] - m) / z);"),
     "renorm_wrong_index": ("w[j] = (exp(logits_row[ids[j]] - m) / z) / ps;",
                            "w[j] = (exp(logits_row[j] - m) / z) / ps;"),
+    "cache_weights_from_biased_logits": ("w[t * k + j] = (exp(z[id[j]] - zmax) / zsum) / ps;",
+                                         "w[t * k + j] = (exp(zb[id[j]] - zmax) / zsum) / ps;"),
+    "cache_delta_is_max_only": ("const double delta = zmax - zmin;", "const double delta = zmax;"),
+    "cache_bias_sign": ("zb[e] = z[e] + lambda * delta * (cached[e] ? 1.0 : 0.0);",
+                        "zb[e] = z[e] - lambda * delta * (cached[e] ? 1.0 : 0.0);"),
     "scale_group_index": ("double s = bf16_bits_to_double(scale[n * (K / 32) + c / 32]);",
                           "double s = bf16_bits_to_double(scale[n * (K / 32) + (c / 32 + 1) % (K / 32)]);"),
 }
@@ -48,6 +54,7 @@ def test_pins_catch_planted_mistake(name, tmp_path):
                            "-o", str(so), "-lm"])
     env = dict(os.environ, ORACLE_LIB=str(so), OMP_NUM_THREADS="2")
     r = subprocess.run([sys.executable, "-m", "pytest", "-x", "-q", "-p", "no:cacheprovider",
-                        os.path.join(ROOT, "tests", "test_oracle_pins.py")],
+                        os.path.join(ROOT, "tests", "test_oracle_pins.py"),
+                        os.path.join(ROOT, "tests", "test_oracle_cache_route.py")],
                        cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
     assert r.returncode != 0, f"pins did not catch mutant {name}:\n{r.stdout[-2000:]}"
