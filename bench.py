@@ -9,6 +9,7 @@ Workloads (synthetic seeded layers of the Qwen3-Next-80B-A3B MoE shape: hidden 2
               12 distinct layers (38.7 GB), so no step finds its weights in L2
   fewrow_t2 / fewrow_t3   a 12-layer bf16 stack of independent layers, 2 or 3 tokens
   int4_48     a 48-layer int4 group-32 stack, one token
+  int2_48     a 48-layer int2 group-32 stack (this library's lower-bit format), one token
   prefill     a 2048-token chunk through one bf16 layer with Zipf(1.1) router offsets
 
 One JSON line on rank 0: the device-timed throughput (CUDA events on the launching
@@ -18,7 +19,7 @@ figure through the C ABI with pinned host buffers, the fp64 oracle on the host c
 and the SM clocks seen during the timed region. A step of a stack workload is one token
 (T rows) through the whole stack, so its tokens/s are model-depth tokens. The default
 run (decode_t1) adds one object per other workload (fewrow_t2, fewrow_t3, int4_48,
-prefill, prefill_uniform), each with its own roofline, end-to-end figure and clocks.
+int2_48, prefill, prefill_uniform), each with its own roofline, end-to-end figure and clocks.
 The path does not shard (one layer fits one GPU): with N > 1 every rank runs its own
 replica ("replicas only"), the value is the sum over ranks.
 """
@@ -48,6 +49,7 @@ FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
 QWEN = mi.LayerShape(H=2048, E=512, k=10, I=512, Is=512)
 QWEN_INT4 = mi.LayerShape(H=2048, E=512, k=10, I=512, Is=512, expert_dtype="int4g32")
+QWEN_INT2 = mi.LayerShape(H=2048, E=512, k=10, I=512, Is=512, expert_dtype="int2g32")
 QWEN_ZIPF = mi.LayerShape(H=2048, E=512, k=10, I=512, Is=512, zipf_s=1.1)
 
 WORKLOADS = {
@@ -59,6 +61,8 @@ WORKLOADS = {
                       desc="12 distinct Qwen3-Next-shaped bf16 layers back to back, T=3"),
     "int4_48": dict(shape=QWEN_INT4, T=1, layers=48, stack=True, seed=4000, kernel="decode_kernel",
                     desc="48 distinct Qwen3-Next-shaped layers, int4 group-32 experts, decode T=1"),
+    "int2_48": dict(shape=QWEN_INT2, T=1, layers=48, stack=True, seed=5000, kernel="decode1_kernel",
+                    desc="48 distinct Qwen3-Next-shaped layers, int2 group-32 experts, decode T=1"),
     "prefill": dict(shape=QWEN_ZIPF, T=2048, layers=1, stack=False, seed=3000, kernel="layer (4 kernels)",
                     desc="Qwen3-Next-shaped MoE layer, bf16, 2048-token prefill chunk, Zipf(1.1) router offsets"),
     # the same chunk with unbiased routing: every expert is touched, so the step streams all
@@ -83,19 +87,22 @@ def peaks():
     return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, 1400.0, "fallback"
 
 
-def expert_bytes(shape):
-    """Bytes of one expert's three matrices (int4: packed codes + bf16 scales)."""
-    H, I = shape.H, shape.I
-    if shape.expert_dtype == "int4g32":
+def _matrix_bytes(dtype, H, I):
+    """Bytes of one expert's three H x I matrices (packed types: codes + bf16 group scales)."""
+    if dtype == "int4g32":
         return 3 * (H * I // 2 + H * I // 32 * 2)
-    return 3 * H * I * (4 if shape.expert_dtype == "f32" else 2)
+    if dtype == "int2g32":
+        return 3 * (H * I // 4 + H * I // 32 * 2)
+    return 3 * H * I * (4 if dtype == "f32" else 2)
+
+
+def expert_bytes(shape):
+    """Bytes of one routed expert's three matrices."""
+    return _matrix_bytes(shape.expert_dtype, shape.H, shape.I)
 
 
 def shared_bytes(shape):
-    H, I = shape.H, shape.Is
-    if shape.expert_dtype == "int4g32":
-        return 3 * (H * I // 2 + H * I // 32 * 2)
-    return 3 * H * I * (4 if shape.expert_dtype == "f32" else 2)
+    return _matrix_bytes(shape.expert_dtype, shape.H, shape.Is)
 
 
 def layer_call_bytes(shape, T, distinct):
@@ -509,7 +516,7 @@ def gpu_arm(args, wl, world, rank, local, B=None, name=None):
     result = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K, "warmup": W,
         "ms_per_step": el_ms / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "bf16" if shape.expert_dtype == "bf16" else ("int4g32" if shape.expert_dtype == "int4g32" else "f32"),
+        "dtype": shape.expert_dtype,
         "data": "synthetic",
         "config": {"workload": wl["desc"], "tokens_per_step": tokens_per_step, "layers": wl["layers"],
                    "layers_per_step": wl["layers"] if wl["stack"] else 1,
@@ -577,8 +584,59 @@ def e2e_arm(args, wl, smg, B, stream, world):
                    "host wall clock around the K steps"}
 
 
-SUB_WORKLOADS = ("fewrow_t2", "fewrow_t3", "int4_48", "prefill", "prefill_uniform")
-SUB_STEPS = {"fewrow_t2": 200, "fewrow_t3": 200, "int4_48": 100, "prefill": 50, "prefill_uniform": 30}
+MIDBATCH_T = (1, 2, 3, 4, 5, 8, 16, 32, 64, 128, 256)
+
+
+def midbatch_sweep(args, world, rank, local):
+    """Per-call time of one bf16 layer at T = 1 .. 256 on a rotation of 12 distinct layers
+    (inputs larger than L2): the decode kernels serve T <= 4, the batched tensor-core path
+    T > 4. Reports, per T, the device time per call (CUDA events around a CUDA graph of the
+    timed calls), the distinct experts touched, the algorithmic bytes and their rate."""
+    import sparse_moe_gemv_b200 as smg
+    smg.load()
+    wl = dict(WORKLOADS["decode_t1"])
+    shape, nl = wl["shape"], wl["layers"]
+    tens = [mi.make_layer(shape, wl["seed"] + l, "cuda") for l in range(nl)]
+    hbm, bf16, _, src = peaks()
+    rows = []
+    for T in MIDBATCH_T:
+        twl = dict(wl, T=T)
+        B = build_workload(twl, smg, tens=tens)
+        stream = torch.cuda.Stream()
+        step, _ = make_step(twl, smg, B, stream)
+        with torch.cuda.stream(stream):
+            step(0)
+        torch.cuda.synchronize()
+        reps = max(2, min(args.steps, 240) // nl)
+        runner = GraphRunner(step, nl, stream)
+        runner.prepare(nl * reps)
+        with torch.cuda.stream(stream):
+            runner.run(nl * 2)
+        torch.cuda.synchronize()
+        ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            ev0.record(stream)
+            runner.run(nl * reps)
+            ev1.record(stream)
+        torch.cuda.synchronize()
+        smg.redmoe_check_timeout(B["work"], stream=stream)
+        us = ev0.elapsed_time(ev1) * 1e3 / (nl * reps)
+        distinct = distinct_experts(B)
+        nbytes = statistics.mean(layer_call_bytes(shape, T, d) for d in distinct)
+        rows.append({"T": T, "path": "decode" if T <= 4 else "batched", "us_per_call": us,
+                     "tokens_per_s": T / us * 1e6, "distinct_experts": statistics.mean(distinct),
+                     "bytes_per_call": nbytes, "gbs": nbytes / us / 1e3, "hbm_frac": nbytes / us / 1e3 / hbm,
+                     "tflops": layer_flops(shape, T) / us / 1e6})
+        B.clear()
+        torch.cuda.synchronize()
+    return {"metric": METRIC, "workload": "midbatch", "unit": "us per layer call",
+            "config": {"workload": wl["desc"].replace("decode T=1", "T = 1..256"), "layers_in_rotation": nl,
+                       "peak_source": src},
+            "rows": rows}
+
+
+SUB_WORKLOADS = ("fewrow_t2", "fewrow_t3", "int4_48", "int2_48", "prefill", "prefill_uniform")
+SUB_STEPS = {"fewrow_t2": 200, "fewrow_t3": 200, "int4_48": 100, "int2_48": 100, "prefill": 50, "prefill_uniform": 30}
 
 
 def sub_result(res):
@@ -601,7 +659,7 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=20000)
     ap.add_argument("--warmup", type=int, default=240)
-    ap.add_argument("--workload", default="decode_t1", choices=sorted(WORKLOADS))
+    ap.add_argument("--workload", default="decode_t1", choices=sorted(WORKLOADS) + ["midbatch"])
     ap.add_argument("--impl", default="redmoe", choices=["redmoe", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extra", action="store_true",
@@ -611,10 +669,17 @@ def main():
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
+    world, rank, local = dist_setup()
+    if args.workload == "midbatch":
+        res = midbatch_sweep(args, world, rank, local)
+        if rank == 0:
+            print(json.dumps(res), flush=True)
+        if world > 1:
+            torch.distributed.destroy_process_group()
+        return
     wl = dict(WORKLOADS[args.workload])
     if args.layers:
         wl["layers"] = args.layers
-    world, rank, local = dist_setup()
     if args.impl == "reference":
         res = reference_arm(args, wl, world, rank)
         if rank == 0:

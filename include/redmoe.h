@@ -59,8 +59,14 @@ typedef enum {
  * packed bytes [N, K/2] (element 2b in the low nibble of byte b, 2b+1 in the high
  * nibble, nibble = code + 8, codes -8..7) plus bf16 scales [N, K/32], one per 32
  * consecutive elements of a row; element value = scale * (nibble - 8). This format is
- * defined by this library (the pages ship GGUF IQ types only). */
-typedef enum { REDMOE_F32 = 0, REDMOE_BF16 = 1, REDMOE_INT4G32 = 2 } redmoe_dtype;
+ * defined by this library (the pages ship GGUF IQ types only).
+ * REDMOE_INT2G32 (expert weights only), this library's lower-bit counterpart (the pages
+ * ship 2-bit expert files, guide "DwarfStar Red Lite", "Measured performance"): [N, K]
+ * is stored as packed bytes [N, K/4] (elements 4b .. 4b+3 in bits 0-1, 2-3, 4-5, 6-7 of
+ * byte b, code = q + 2, codes 0..3) plus bf16 scales [N, K/32]; element value =
+ * scale * (code - 2). Supported at one token row (T = 1) with hidden 2048 and expert
+ * intermediate 512; other sizes return REDMOE_ERR_UNSUPPORTED. */
+typedef enum { REDMOE_F32 = 0, REDMOE_BF16 = 1, REDMOE_INT4G32 = 2, REDMOE_INT2G32 = 3 } redmoe_dtype;
 
 /* One MoE layer. All tensors device-resident, row-major; E = n_experts, H = hidden,
  * I = inter, Is = shared_inter. The routed expert stacks keep the expert as the
@@ -78,18 +84,18 @@ typedef struct redmoe_layer {
     const void *router_w;        /* [E, H]                                                    */
     const float *router_bias;    /* [E] fp32 per-expert logit offset, or NULL                 */
     const void *shared_gate_w;   /* [H]                                                       */
-    const void *w_gate;          /* [E, I, H]   (int4: u8 [E, I, H/2])                        */
-    const void *w_up;            /* [E, I, H]   (int4: u8 [E, I, H/2])                        */
-    const void *w_down;          /* [E, H, I]   (int4: u8 [E, H, I/2])                        */
-    const void *s_gate;          /* int4: bf16 [E, I, H/32], 16-byte aligned; otherwise NULL  */
-    const void *s_up;            /* int4: bf16 [E, I, H/32]                                   */
-    const void *s_down;          /* int4: bf16 [E, H, I/32]                                   */
-    const void *sh_gate;         /* [Is, H]     (int4: u8 [Is, H/2])                          */
+    const void *w_gate;          /* [E, I, H]   (int4: u8 [E, I, H/2]; int2: u8 [E, I, H/4])  */
+    const void *w_up;            /* [E, I, H]   (as w_gate)                                   */
+    const void *w_down;          /* [E, H, I]   (int4: u8 [E, H, I/2]; int2: u8 [E, H, I/4])  */
+    const void *s_gate;          /* int4/int2: bf16 [E, I, H/32], 16-byte aligned; else NULL  */
+    const void *s_up;            /* int4/int2: bf16 [E, I, H/32]                              */
+    const void *s_down;          /* int4/int2: bf16 [E, H, I/32]                              */
+    const void *sh_gate;         /* [Is, H]     (packed like the routed experts)              */
     const void *sh_up;           /* [Is, H]                                                   */
-    const void *sh_down;         /* [H, Is]     (int4: u8 [H, Is/2])                          */
-    const void *sh_s_gate;       /* int4: bf16 [Is, H/32]; otherwise NULL                     */
-    const void *sh_s_up;         /* int4: bf16 [Is, H/32]                                     */
-    const void *sh_s_down;       /* int4: bf16 [H, Is/32]                                     */
+    const void *sh_down;         /* [H, Is]                                                   */
+    const void *sh_s_gate;       /* int4/int2: bf16 [Is, H/32]; otherwise NULL                */
+    const void *sh_s_up;         /* int4/int2: bf16 [Is, H/32]                                */
+    const void *sh_s_down;       /* int4/int2: bf16 [H, Is/32]                                */
 } redmoe_layer;
 
 /* Optional device outputs of the token->expert grouping (see redmoe_route_build). */
@@ -135,6 +141,27 @@ redmoe_status redmoe_workspace_init(void *workspace, size_t workspace_bytes, voi
 redmoe_status redmoe_forward(const redmoe_layer *L, const void *x, int32_t T, float *out,
                              int32_t *topk_ids, float *topk_w, void *workspace,
                              size_t workspace_bytes, const redmoe_route_debug *dbg, void *stream);
+
+/* redmoe_forward with the opt-in cache-aware routing bias of "Research notes, October
+ * 2026", section 4 ("Cache-aware routing bias (z + lambda * Delta * cached)", opt-in
+ * only because it changes outputs). For a caller that keeps only some experts in a
+ * fast tier and wants tokens to prefer those. The pages give only the expression; this
+ * library's reading of it, which the oracle shares:
+ *   cached   [E] uint8 device array: nonzero if the expert is resident in the caller's
+ *            cache;
+ *   lambda   >= 0 (finite); 0 gives exactly the routing of redmoe_forward;
+ *   Delta    the token's logit range, max_e z[e] - min_e z[e] (router offsets included),
+ *            which makes lambda dimensionless: with lambda > 1 and at least k cached
+ *            experts only cached experts are selected;
+ *   ids      the k largest z[e] + lambda * Delta * cached[e], ties to the lower id,
+ *            ordered by that biased logit;
+ *   weights  the softmax of the unbiased logits over all experts, restricted to the
+ *            selection and renormalised (the bias changes which experts run, not how
+ *            their outputs are mixed).
+ * Other arguments, sizes and errors as redmoe_forward (no grouping debug output). */
+redmoe_status redmoe_forward_cached(const redmoe_layer *L, const void *x, int32_t T, float *out,
+                                    int32_t *topk_ids, float *topk_w, const uint8_t *cached, float lambda,
+                                    void *workspace, size_t workspace_bytes, void *stream);
 
 /* The router stage alone: logits, top-k ids, renormalised weights, shared gate.
  *   topk_ids [T, k] int32, topk_w [T, k] fp32, shared_gate [T] fp32 = sigmoid(x . g),

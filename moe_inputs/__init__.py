@@ -19,13 +19,13 @@ name               shape            dtype
 router_w           [E, H]           f32 | bf16
 router_bias        [E]              f32, or None (prefill Zipf workload only)
 shared_gate_w      [H]              same dtype as router_w
-w_gate, w_up       [E, I, H]        f32 | bf16 | u8 packed int4 [E, I, H/2]
-w_down             [E, H, I]        f32 | bf16 | u8 packed int4 [E, H, I/2]
-s_gate, s_up       [E, I, H/32]     bf16 scales (int4 only)
-s_down             [E, H, I/32]     bf16 scales (int4 only)
+w_gate, w_up       [E, I, H]        f32 | bf16 | u8 packed int4 [E, I, H/2] | int2 [E, I, H/4]
+w_down             [E, H, I]        f32 | bf16 | u8 packed int4 [E, H, I/2] | int2 [E, H, I/4]
+s_gate, s_up       [E, I, H/32]     bf16 scales (int4 / int2 only)
+s_down             [E, H, I/32]     bf16 scales (int4 / int2 only)
 sh_gate, sh_up     [Is, H]          expert dtype (packed like the routed experts)
 sh_down            [H, Is]          expert dtype
-sh_s_*             [..., K/32]      bf16 scales (int4 only)
+sh_s_*             [..., K/32]      bf16 scales (int4 / int2 only)
 =================  ===============  ==========================================
 
 int4 group-32 storage format (defined here; the pages ship GGUF IQ formats only):
@@ -35,6 +35,14 @@ per row and per group of 32 consecutive K elements, scale ``s = bf16(amax / 7)``
 Byte ``b`` of a row holds element ``2b`` in its low nibble and ``2b + 1`` in its
 high nibble. A reader recovers ``float(s) * (nibble - 8)``. Quantisation is input
 generation: the kernels and the oracle read the same packed bytes.
+
+int2 group-32 storage format (also defined here; the lower-bit counterpart of int4 g32,
+after the 2-bit expert files the pages ship): per row and per group of 32 consecutive K
+elements, scale ``s = bf16(amax / 1)``, codes ``q = clamp(round_half_even(w / float(s)),
+-1, 1)`` (``q = 0`` when ``s == 0``) computed in fp32, stored as the 2-bit code ``q + 2``.
+Byte ``b`` of a row holds elements ``4b, 4b+1, 4b+2, 4b+3`` in bits 0-1, 2-3, 4-5 and 6-7.
+A reader recovers ``float(s) * (code - 2)`` (code 0, which the quantiser never writes,
+reads as -2).
 """
 
 from __future__ import annotations
@@ -46,7 +54,7 @@ from typing import Dict, Optional
 import numpy as np
 import torch
 
-DTYPES = ("f32", "bf16", "int4g32")
+DTYPES = ("f32", "bf16", "int4g32", "int2g32")
 
 
 @dataclasses.dataclass(frozen=True)
@@ -126,21 +134,45 @@ def quantize_int4g32(w: torch.Tensor):
     return packed, s.contiguous()
 
 
+def quantize_int2g32(w: torch.Tensor):
+    """Pack an fp32 matrix [..., N, K] into the int2 group-32 format described above.
+
+    Returns (packed u8 [..., N, K/4], scales bf16 [..., N, K/32]).
+    """
+    K = w.shape[-1]
+    if K % 32:
+        raise ValueError("K must be a multiple of 32 for int2 group-32")
+    grp = w.reshape(*w.shape[:-1], K // 32, 32)
+    amax = grp.abs().amax(dim=-1)
+    s = amax.to(torch.bfloat16)
+    sf = s.to(torch.float32).unsqueeze(-1)
+    safe = torch.where(sf == 0, torch.ones_like(sf), sf)
+    q = torch.round(grp / safe).clamp_(-1, 1)
+    q = torch.where(sf == 0, torch.zeros_like(q), q)
+    u = (q + 2).to(torch.uint8).reshape(*w.shape[:-1], K)
+    packed = (u[..., 0::4] | (u[..., 1::4] << 2) | (u[..., 2::4] << 4) | (u[..., 3::4] << 6)).contiguous()
+    return packed, s.contiguous()
+
+
+QUANTIZERS = {"int4g32": (quantize_int4g32, 2), "int2g32": (quantize_int2g32, 4)}  # (packer, elements per byte)
+
+
 def _expert_tensor(shape, sigma, dtype, g, device, chunk=64):
     """Draw [E, N, K] weights expert-chunk by expert-chunk (bounded fp32 temporaries)."""
     E, N, K = shape
-    if dtype != "int4g32":
+    if dtype not in QUANTIZERS:
         tdt = torch.float32 if dtype == "f32" else torch.bfloat16
         out = torch.empty(E, N, K, dtype=tdt, device=device)
         for e0 in range(0, E, chunk):
             e1 = min(E, e0 + chunk)
             out[e0:e1] = _store(_normal((e1 - e0, N, K), sigma, g, device), dtype)
         return out, None
-    packed = torch.empty(E, N, K // 2, dtype=torch.uint8, device=device)
+    quant, per_byte = QUANTIZERS[dtype]
+    packed = torch.empty(E, N, K // per_byte, dtype=torch.uint8, device=device)
     scales = torch.empty(E, N, K // 32, dtype=torch.bfloat16, device=device)
     for e0 in range(0, E, chunk):
         e1 = min(E, e0 + chunk)
-        p, s = quantize_int4g32(_normal((e1 - e0, N, K), sigma, g, device))
+        p, s = quant(_normal((e1 - e0, N, K), sigma, g, device))
         packed[e0:e1] = p
         scales[e0:e1] = s
     return packed, scales

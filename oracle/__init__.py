@@ -22,7 +22,7 @@ import numpy as np
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "moe_oracle.c")
 _LIB = os.path.join(_HERE, "liboracle.so")
-_DT = {"f32": 0, "bf16": 1, "int4g32": 2}
+_DT = {"f32": 0, "bf16": 1, "int4g32": 2, "int2g32": 3}
 _lock = threading.Lock()
 _handle = None
 
@@ -68,6 +68,7 @@ def _lib():
             lib.orc_expert_ffn.argtypes = [P, i32, P, P]
             lib.orc_route_build.argtypes = [i32, i32, i32, P, P, P, P]
             lib.orc_dequant_int4.argtypes = [i32, i32, P, P, P]
+            lib.orc_dequant_int2.argtypes = [i32, i32, P, P, P]
             lib.orc_renorm.argtypes = [i32, i32, P, P, P]
             lib.orc_cache_route.argtypes = [i32, i32, i32, P, P, C.c_double, P, P, P]
             lib.orc_num_threads.argtypes = []
@@ -250,6 +251,16 @@ def dequant_int4(packed, scales):
     N, K = packed.shape[0], packed.shape[1] * 2
     out = np.zeros((N, K), np.float64)
     _check(_lib().orc_dequant_int4(N, K, _ptr(packed), _ptr(scales), _ptr(out)))
+    return out
+
+
+def dequant_int2(packed, scales):
+    """Dequantise an int2 group-32 matrix (packed u8 [N, K/4], scales bf16 bits [N, K/32])."""
+    packed = np.ascontiguousarray(packed, np.uint8)
+    scales = np.ascontiguousarray(scales, np.uint16)
+    N, K = packed.shape[0], packed.shape[1] * 4
+    out = np.zeros((N, K), np.float64)
+    _check(_lib().orc_dequant_int2(N, K, _ptr(packed), _ptr(scales), _ptr(out)))
     return out
 
 

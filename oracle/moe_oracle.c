@@ -54,7 +54,7 @@
 #include <omp.h>
 #endif
 
-enum { ORC_F32 = 0, ORC_BF16 = 1, ORC_INT4G32 = 2 };
+enum { ORC_F32 = 0, ORC_BF16 = 1, ORC_INT4G32 = 2, ORC_INT2G32 = 3 };
 
 enum {
     ORC_OK = 0,
@@ -88,6 +88,12 @@ static double bf16_bits_to_double(uint16_t b)
     return (double)f;
 }
 
+/* Scale of the 32-element group holding element (n, c) of a packed N x K matrix. */
+static double group_scale(const uint16_t *scale, long K, long n, long c)
+{
+    return bf16_bits_to_double(scale[n * (K / 32) + c / 32]);
+}
+
 /* Element (n, c) of an N x K matrix stored in `dtype`. */
 static double w_at(const void *w, const uint16_t *scale, int dtype, long K, long n, long c)
 {
@@ -96,11 +102,15 @@ static double w_at(const void *w, const uint16_t *scale, int dtype, long K, long
         return (double)((const float *)w)[n * K + c];
     case ORC_BF16:
         return bf16_bits_to_double(((const uint16_t *)w)[n * K + c]);
+    case ORC_INT2G32: {
+        uint8_t byte = ((const uint8_t *)w)[n * (K / 4) + c / 4];
+        int code = (byte >> (2 * (c % 4))) & 3;
+        return group_scale(scale, K, n, c) * (double)(code - 2);
+    }
     default: {
         uint8_t byte = ((const uint8_t *)w)[n * (K / 2) + c / 2];
         int nibble = (c & 1) ? (byte >> 4) : (byte & 15);
-        double s = bf16_bits_to_double(scale[n * (K / 32) + c / 32]);
-        return s * (double)(nibble - 8);
+        return group_scale(scale, K, n, c) * (double)(nibble - 8);
     }
     }
 }
@@ -112,9 +122,9 @@ static double act_at(const void *x, int dtype, long i)
     return bf16_bits_to_double(((const uint16_t *)x)[i]);
 }
 
-static int dtype_ok(int d, int allow_int4)
+static int dtype_ok(int d, int allow_packed)
 {
-    return d == ORC_F32 || d == ORC_BF16 || (allow_int4 && d == ORC_INT4G32);
+    return d == ORC_F32 || d == ORC_BF16 || (allow_packed && (d == ORC_INT4G32 || d == ORC_INT2G32));
 }
 
 static int shape_ok(const orc_layer *L)
@@ -123,7 +133,7 @@ static int shape_ok(const orc_layer *L)
         return 0;
     if (!dtype_ok(L->x_dtype, 0) || !dtype_ok(L->router_dtype, 0) || !dtype_ok(L->expert_dtype, 1))
         return 0;
-    if (L->expert_dtype == ORC_INT4G32 && (L->H % 32 || L->I % 32 || L->Is % 32))
+    if ((L->expert_dtype == ORC_INT4G32 || L->expert_dtype == ORC_INT2G32) && (L->H % 32 || L->I % 32 || L->Is % 32))
         return 0;
     return 1;
 }
@@ -156,6 +166,18 @@ int orc_dequant_int4(int32_t N, int32_t K, const uint8_t *packed, const uint16_t
     for (long n = 0; n < N; ++n)
         for (long c = 0; c < K; ++c)
             out[n * K + c] = w_at(packed, scales, ORC_INT4G32, K, n, c);
+    return ORC_OK;
+}
+
+/* int2 group-32: element c of row n is scale[n][c/32] * (code - 2), the 2-bit code in
+ * bits 2*(c%4) .. 2*(c%4)+1 of byte c/4. */
+int orc_dequant_int2(int32_t N, int32_t K, const uint8_t *packed, const uint16_t *scales, double *out)
+{
+    if (N < 0 || K <= 0 || K % 32 || !packed || !scales || !out)
+        return ORC_ERR_ARG;
+    for (long n = 0; n < N; ++n)
+        for (long c = 0; c < K; ++c)
+            out[n * K + c] = w_at(packed, scales, ORC_INT2G32, K, n, c);
     return ORC_OK;
 }
 

@@ -7,7 +7,8 @@ and has no fallback: if the library is missing it raises.
 Names match the C entry points (redmoe_forward, redmoe_router, redmoe_route_build,
 redmoe_forward_stack, redmoe_forward_noalloc, redmoe_workspace_bytes,
 redmoe_workspace_init, redmoe_check_timeout, redmoe_selftest_wait_limit,
-redmoe_fill_shared_memory, redmoe_status_string, redmoe_abi_version).
+redmoe_fill_shared_memory, redmoe_forward_cached, redmoe_status_string,
+redmoe_abi_version).
 """
 
 from __future__ import annotations
@@ -22,14 +23,14 @@ import torch
 _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libredmoe.so")
 ABI_VERSION = 1
-DTYPES = {"f32": 0, "bf16": 1, "int4g32": 2}
+DTYPES = {"f32": 0, "bf16": 1, "int4g32": 2, "int2g32": 3}
 STATUS = {0: "REDMOE_OK", 1: "REDMOE_ERR_INVALID_ARG", 2: "REDMOE_ERR_UNSUPPORTED", 3: "REDMOE_ERR_WORKSPACE",
           4: "REDMOE_ERR_CUDA", 5: "REDMOE_ERR_TIMEOUT"}
 # entry points declared in include/redmoe.h
 SYMBOLS = ("redmoe_abi_version", "redmoe_status_string", "redmoe_workspace_bytes", "redmoe_workspace_init",
            "redmoe_forward", "redmoe_router", "redmoe_route_build", "redmoe_forward_stack",
            "redmoe_check_timeout", "redmoe_forward_noalloc", "redmoe_selftest_wait_limit",
-           "redmoe_fill_shared_memory")
+           "redmoe_fill_shared_memory", "redmoe_forward_cached")
 
 _lock = threading.Lock()
 _lib = None
@@ -90,6 +91,8 @@ def load():
         lib.redmoe_forward_noalloc.argtypes = [P, P, i32, P, P, P, P]
         lib.redmoe_selftest_wait_limit.restype = i32
         lib.redmoe_selftest_wait_limit.argtypes = [P, sz, i32, C.c_uint64, P]
+        lib.redmoe_forward_cached.restype = i32
+        lib.redmoe_forward_cached.argtypes = [P, P, i32, P, P, P, P, C.c_float, P, sz, P]
         lib.redmoe_fill_shared_memory.restype = i32
         lib.redmoe_fill_shared_memory.argtypes = [C.c_uint32, P]
         if lib.redmoe_abi_version() != ABI_VERSION:
@@ -187,6 +190,18 @@ def redmoe_forward(layer: Layer, x: torch.Tensor, out: torch.Tensor, topk_ids: t
                             _ptr(workspace), workspace.numel() * workspace.element_size(),
                             None if dbg_s is None else C.byref(dbg_s), _stream(stream))
     _check(st, "redmoe_forward")
+
+
+def redmoe_forward_cached(layer: Layer, x: torch.Tensor, out: torch.Tensor, topk_ids: torch.Tensor,
+                          topk_w: torch.Tensor, cached: torch.Tensor, lam: float, workspace: torch.Tensor,
+                          stream=None) -> None:
+    """redmoe_forward with the opt-in cache-aware routing bias: cached [E] uint8 device mask
+    of experts resident in the caller's cache, lam >= 0 (0: plain routing)."""
+    T = x.shape[0]
+    st = load().redmoe_forward_cached(layer.ref, _ptr(x), int(T), _ptr(out), _ptr(topk_ids), _ptr(topk_w),
+                                      _ptr(cached), float(lam), _ptr(workspace),
+                                      workspace.numel() * workspace.element_size(), _stream(stream))
+    _check(st, "redmoe_forward_cached")
 
 
 def redmoe_router(layer: Layer, x: torch.Tensor, topk_ids: torch.Tensor, topk_w: torch.Tensor,

@@ -43,7 +43,7 @@ namespace {
 
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
-int elems_per_chunk(int dt) { return dt == DT_F32 ? 4 : (dt == DT_BF16 ? 8 : 32); }
+int elems_per_chunk(int dt) { return dt == DT_F32 ? 4 : (dt == DT_BF16 ? 8 : (dt == DT_INT4 ? 32 : 64)); }
 
 // Workspace carve-up of the router entry point and of the batched path.
 struct BatchWs {
@@ -89,10 +89,10 @@ redmoe_status check_layer(const redmoe_layer* L) {
     if (H <= 0 || E <= 0 || k <= 0 || I <= 0 || Is <= 0) return REDMOE_ERR_INVALID_ARG;
     if (k > E || k > MAX_TOPK || E > MAX_EXPERTS) return REDMOE_ERR_INVALID_ARG;
     const int xt = L->x_dtype, rt = L->router_dtype, wt = L->expert_dtype;
-    if (xt < 0 || xt > 2 || rt < 0 || rt > 2 || wt < 0 || wt > 2) return REDMOE_ERR_INVALID_ARG;
-    if (xt == DT_INT4 || rt == DT_INT4) return REDMOE_ERR_INVALID_ARG;
+    if (xt < 0 || xt > 3 || rt < 0 || rt > 3 || wt < 0 || wt > 3) return REDMOE_ERR_INVALID_ARG;
+    if (xt == DT_INT4 || rt == DT_INT4 || xt == DT_INT2 || rt == DT_INT2) return REDMOE_ERR_INVALID_ARG;
     const bool combo = (xt == DT_F32 && rt == DT_F32 && wt == DT_F32) ||
-                       (xt == DT_BF16 && rt == DT_BF16 && (wt == DT_BF16 || wt == DT_INT4));
+                       (xt == DT_BF16 && rt == DT_BF16 && (wt == DT_BF16 || wt == DT_INT4 || wt == DT_INT2));
     if (!combo) return REDMOE_ERR_UNSUPPORTED;
     // every row is read in 16-byte chunks; int4 rows also in whole scale groups
     if (H % 32 || I % 32 || Is % 32) return REDMOE_ERR_INVALID_ARG;
@@ -103,7 +103,7 @@ redmoe_status check_layer(const redmoe_layer* L) {
     if (L->router_bias && !aligned(L->router_bias, 4)) return REDMOE_ERR_INVALID_ARG;
     const void* sc[] = {L->s_gate, L->s_up, L->s_down, L->sh_s_gate, L->sh_s_up, L->sh_s_down};
     for (const void* p : sc) {
-        if (wt == DT_INT4) {
+        if (wt == DT_INT4 || wt == DT_INT2) {
             if (!p || !aligned(p, 16)) return REDMOE_ERR_INVALID_ARG;
         }
     }
@@ -195,6 +195,28 @@ redmoe_status redmoe_forward(const redmoe_layer* L, const void* x, int32_t T, fl
         st = launch_route_build(topk_ids, T, L->top_k, L->n_experts, dbg->counts, dbg->offsets, dbg->perm, 0,
                                 nullptr, s, nullptr);
     return st;
+}
+
+redmoe_status redmoe_forward_cached(const redmoe_layer* L, const void* x, int32_t T, float* out, int32_t* topk_ids,
+                                    float* topk_w, const uint8_t* cached, float lambda, void* workspace,
+                                    size_t workspace_bytes, void* stream) {
+    redmoe_status st = check_layer(L);
+    if (st != REDMOE_OK) return st;
+    if (T < 0 || !(lambda >= 0.0f) || !(lambda <= 3.0e38f)) return REDMOE_ERR_INVALID_ARG;
+    if (T == 0) return REDMOE_OK;
+    if (!x || !out || !topk_ids || !topk_w || !cached) return REDMOE_ERR_INVALID_ARG;
+    if (!aligned(x, 16) || !aligned(out, 16) || !aligned(topk_ids, 4) || !aligned(topk_w, 4))
+        return REDMOE_ERR_INVALID_ARG;
+    if ((st = check_ws(L, T, workspace, workspace_bytes)) != REDMOE_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const CacheBias cb{cached, lambda};
+    if (T > DECODE_MAX_T) {
+        if (!batch_shape_ok(L)) return REDMOE_ERR_UNSUPPORTED;
+        if ((long long)T * L->top_k + T > (1ll << 30)) return REDMOE_ERR_INVALID_ARG;
+        return launch_batched(L, x, T, out, topk_ids, topk_w, workspace, nullptr, s, nullptr, cb);
+    }
+    const DecLayer d = dec_layer(L, x, out, topk_ids, topk_w);
+    return launch_decode(L, &d, 1, T, workspace, s, nullptr, cb);
 }
 
 redmoe_status redmoe_router(const redmoe_layer* L, const void* x, int32_t T, int32_t* topk_ids, float* topk_w,

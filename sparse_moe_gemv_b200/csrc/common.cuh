@@ -6,7 +6,7 @@
 
 namespace redmoe {
 
-enum : int { DT_F32 = 0, DT_BF16 = 1, DT_INT4 = 2 };
+enum : int { DT_F32 = 0, DT_BF16 = 1, DT_INT4 = 2, DT_INT2 = 3 };
 
 // Bits of the workspace error word.
 enum : int { ERRBIT_TIMEOUT = 1 };
@@ -45,12 +45,24 @@ __device__ __forceinline__ float key_to_float(uint32_t k) {
     return __uint_as_float(u);
 }
 
+// int2 codes n and n+1 of w as floats (code - 2): exponent-trick conversion, exact.
+__device__ __forceinline__ float2 crumb2(uint32_t w, int n) {
+    const float a = __uint_as_float(0x4B000000u | ((w >> (2 * n)) & 3u));
+    const float b = __uint_as_float(0x4B000000u | ((w >> (2 * n + 2)) & 3u));
+    return __fadd2_rn(make_float2(a, b), make_float2(-8388610.0f, -8388610.0f));
+}
+
 // ------------------------------------------------------------------- loads
 // Streaming read-only 16-byte load: weights are read once per call, keep them out of L1.
 __device__ __forceinline__ uint4 ld_stream(const void* p) {
     uint4 v;
     asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
                  : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(p));
+    return v;
+}
+__device__ __forceinline__ uint32_t ld_stream_u32(const void* p) {
+    uint32_t v;
+    asm volatile("ld.global.nc.L1::no_allocate.u32 %0, [%1];" : "=r"(v) : "l"(p));
     return v;
 }
 __device__ __forceinline__ uint16_t ld_stream_u16(const void* p) {

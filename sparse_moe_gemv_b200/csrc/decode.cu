@@ -246,6 +246,7 @@ struct DecParams {
     float* hsh;      // 2 x [T, Is]
     float* hrt;      // [T * k, I]     (slot t*k + j)
     uint64_t timeout_ns;
+    CacheBias cb;
     DecLayer L[NL];
 };
 
@@ -431,9 +432,19 @@ __global__ void __launch_bounds__(THREADS, 1) decode_kernel(const __grid_constan
         grid_barrier(p.ctl, nblocks, bar_idx++, to);
 
         // ---------------------------------------------------------- phase B
-        for (int i = threadIdx.x; i < T * E; i += THREADS) s_keys[i] = order_key(__ldcg(p.logits + i));
-        __syncthreads();
-        if (warp < T) warp_topk_keys(E, k, s_keys + warp * E, s_ids + warp * k, s_w + warp * k);
+        if (p.cb.cached == nullptr) {
+            for (int i = threadIdx.x; i < T * E; i += THREADS) s_keys[i] = order_key(__ldcg(p.logits + i));
+            __syncthreads();
+            if (warp < T) warp_topk_keys(E, k, s_keys + warp * E, s_ids + warp * k, s_w + warp * k);
+        } else if (warp < T) {  // opt-in cache-aware routing
+            int id;
+            float wv;
+            warp_route_any(p.logits + warp * E, E, k, p.cb.cached, p.cb.lambda, id, wv);
+            if (lane < k) {
+                s_ids[warp * k + lane] = id;
+                s_w[warp * k + lane] = wv;
+            }
+        }
         __syncthreads();
         // distinct experts over the T*k routed slots: u numbers the first occurrences in
         // slot order; slot t*k + j of token t maps to u with weight w[t][j]
@@ -695,7 +706,8 @@ int blocks_per_sm(const void* kern, int smem) {
 }
 
 template <int XT, int RT, int WT, int T, int NL>
-redmoe_status launch_one(const redmoe_layer* sh, const DecLayer* layers, int n_layers, void* ws, cudaStream_t stream) {
+redmoe_status launch_one(const redmoe_layer* sh, const DecLayer* layers, int n_layers, void* ws, cudaStream_t stream,
+                         CacheBias cb) {
     DevInfo di;
     if (!get_dev_info(&di)) return REDMOE_ERR_CUDA;
     const int RB = (sh->hidden + di.sm_count - 1) / di.sm_count;
@@ -725,6 +737,7 @@ redmoe_status launch_one(const redmoe_layer* sh, const DecLayer* layers, int n_l
     q.hsh = reinterpret_cast<float*>(base + L.hsh);
     q.hrt = reinterpret_cast<float*>(base + L.hrt);
     q.timeout_ns = BARRIER_TIMEOUT_NS;
+    q.cb = cb;
     for (int i = 0; i < n_layers; ++i) q.L[i] = layers[i];
 
     cudaLaunchConfig_t cfg = {};
@@ -744,16 +757,16 @@ redmoe_status launch_one(const redmoe_layer* sh, const DecLayer* layers, int n_l
 
 template <int XT, int RT, int WT, int T>
 redmoe_status launch_t(const redmoe_layer* sh, const DecLayer* layers, int n_layers, void* ws, cudaStream_t stream,
-                       int* launches) {
+                       int* launches, CacheBias cb) {
     redmoe_status st = REDMOE_OK;
     if (n_layers == 1) {
-        st = launch_one<XT, RT, WT, T, 1>(sh, layers, 1, ws, stream);
+        st = launch_one<XT, RT, WT, T, 1>(sh, layers, 1, ws, stream, cb);
         if (st == REDMOE_OK && launches) *launches += 1;
         return st;
     }
     for (int l0 = 0; l0 < n_layers && st == REDMOE_OK; l0 += MAX_STACK) {
         const int n = n_layers - l0 < MAX_STACK ? n_layers - l0 : MAX_STACK;
-        st = launch_one<XT, RT, WT, T, MAX_STACK>(sh, layers + l0, n, ws, stream);
+        st = launch_one<XT, RT, WT, T, MAX_STACK>(sh, layers + l0, n, ws, stream, cb);
         if (st == REDMOE_OK && launches) *launches += 1;
     }
     return st;
@@ -761,12 +774,12 @@ redmoe_status launch_t(const redmoe_layer* sh, const DecLayer* layers, int n_lay
 
 template <int XT, int RT, int WT>
 redmoe_status launch_dt(const redmoe_layer* sh, const DecLayer* layers, int n_layers, int T, void* ws,
-                        cudaStream_t stream, int* launches) {
+                        cudaStream_t stream, int* launches, CacheBias cb) {
     switch (T) {
-        case 1: return launch_t<XT, RT, WT, 1>(sh, layers, n_layers, ws, stream, launches);
-        case 2: return launch_t<XT, RT, WT, 2>(sh, layers, n_layers, ws, stream, launches);
-        case 3: return launch_t<XT, RT, WT, 3>(sh, layers, n_layers, ws, stream, launches);
-        case 4: return launch_t<XT, RT, WT, 4>(sh, layers, n_layers, ws, stream, launches);
+        case 1: return launch_t<XT, RT, WT, 1>(sh, layers, n_layers, ws, stream, launches, cb);
+        case 2: return launch_t<XT, RT, WT, 2>(sh, layers, n_layers, ws, stream, launches, cb);
+        case 3: return launch_t<XT, RT, WT, 3>(sh, layers, n_layers, ws, stream, launches, cb);
+        case 4: return launch_t<XT, RT, WT, 4>(sh, layers, n_layers, ws, stream, launches, cb);
         default: return REDMOE_ERR_UNSUPPORTED;
     }
 }
@@ -787,6 +800,7 @@ DecodeWs decode_ws_layout(int T, int E, int k, int I, int Is) {
 // Shapes the decode kernel stages: every single weight segment must fit one 4 KiB stage.
 bool decode_shape_ok(const redmoe_layer* sh) {
     const int H = sh->hidden, I = sh->inter, Is = sh->shared_inter, wt = sh->expert_dtype, rt = sh->router_dtype;
+    if (wt == DT_INT2) return false;  // int2 experts: one-row kernel only
     if (row_bytes(rt, H) > SEG_MAX || row_bytes(wt, H) > SEG_MAX) return false;
     if (align16(int(row_bytes(wt, H))) + scale_bytes(wt, H) > SB) return false;
     if (decode_rows_per_stage(sh) < 1) return false;
@@ -795,15 +809,16 @@ bool decode_shape_ok(const redmoe_layer* sh) {
 }
 
 redmoe_status launch_decode(const redmoe_layer* sh, const DecLayer* layers, int n_layers, int T, void* ws,
-                            cudaStream_t stream, int* launches) {
+                            cudaStream_t stream, int* launches, CacheBias cb) {
+    if (T == 1 && decode1_shape_ok(sh)) return launch_decode1(sh, layers, n_layers, ws, stream, launches, cb);
     if (!decode_shape_ok(sh)) return REDMOE_ERR_UNSUPPORTED;
     const int xt = sh->x_dtype, rt = sh->router_dtype, wt = sh->expert_dtype;
     if (xt == DT_F32 && rt == DT_F32 && wt == DT_F32)
-        return launch_dt<DT_F32, DT_F32, DT_F32>(sh, layers, n_layers, T, ws, stream, launches);
+        return launch_dt<DT_F32, DT_F32, DT_F32>(sh, layers, n_layers, T, ws, stream, launches, cb);
     if (xt == DT_BF16 && rt == DT_BF16 && wt == DT_BF16)
-        return launch_dt<DT_BF16, DT_BF16, DT_BF16>(sh, layers, n_layers, T, ws, stream, launches);
+        return launch_dt<DT_BF16, DT_BF16, DT_BF16>(sh, layers, n_layers, T, ws, stream, launches, cb);
     if (xt == DT_BF16 && rt == DT_BF16 && wt == DT_INT4)
-        return launch_dt<DT_BF16, DT_BF16, DT_INT4>(sh, layers, n_layers, T, ws, stream, launches);
+        return launch_dt<DT_BF16, DT_BF16, DT_INT4>(sh, layers, n_layers, T, ws, stream, launches, cb);
     return REDMOE_ERR_UNSUPPORTED;
 }
 

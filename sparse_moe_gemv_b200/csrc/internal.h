@@ -18,6 +18,13 @@ constexpr int ROUTE_MAX_BLOCKS = 256;  // blocks of the batched routing kernel, 
 
 inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
+// Opt-in cache-aware routing: the selection ranks z + lambda * (max z - min z) * cached[e];
+// cached == nullptr is plain routing.
+struct CacheBias {
+    const uint8_t* cached;
+    float lambda;
+};
+
 // One layer as the decode kernel sees it (pointers into caller memory).
 struct DecLayer {
     const void* router_w;
@@ -57,9 +64,15 @@ struct DecodeWs {
 };
 DecodeWs decode_ws_layout(int T, int E, int k, int I, int Is);
 
+// The one-row kernel (T = 1, bf16 or int4 experts of the Qwen3-Next width): which layers
+// it takes, and its launch over n_layers layers.
+bool decode1_shape_ok(const redmoe_layer* sh);
+redmoe_status launch_decode1(const redmoe_layer* sh, const DecLayer* layers, int n_layers, void* ws,
+                             cudaStream_t stream, int* launches, CacheBias cb);
+
 // Launch the persistent decode kernel over n_layers layers (1..MAX_STACK).
 redmoe_status launch_decode(const redmoe_layer* shape, const DecLayer* layers, int n_layers, int T,
-                            void* workspace, cudaStream_t stream, int* launches);
+                            void* workspace, cudaStream_t stream, int* launches, CacheBias cb = CacheBias{nullptr, 0.0f});
 
 // Workspace carve-up of the batched (grouped-GEMM) path (byte offsets from the base).
 struct BatchLayout {
@@ -68,7 +81,8 @@ struct BatchLayout {
 BatchLayout batch_layout(int T, int E, int k, int H, int I);
 bool batch_shape_ok(const redmoe_layer* L);
 redmoe_status launch_batched(const redmoe_layer* L, const void* x, int T, float* out, int32_t* ids, float* w,
-                             void* ws, const redmoe_route_debug* dbg, cudaStream_t s, int* launches);
+                             void* ws, const redmoe_route_debug* dbg, cudaStream_t s, int* launches,
+                             CacheBias cb = CacheBias{nullptr, 0.0f});
 
 // Device attributes cached per device.
 struct DevInfo {

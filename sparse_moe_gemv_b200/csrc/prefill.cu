@@ -33,7 +33,7 @@ redmoe_status gemm_scatter(GemmParams& p, cudaStream_t s);
 redmoe_status launch_route(const redmoe_layer* L, const void* x, int T, const float* logits, int32_t* ids, float* w,
                            float* sgate, int32_t* counts, int32_t* offsets, int32_t* perm, int tile_m,
                            int32_t* tiles, void* xg, int32_t* bhist, Control* ctl, cudaStream_t stream,
-                           int* launches);
+                           int* launches, CacheBias cb);
 
 BatchLayout batch_layout(int T, int E, int k, int H, int I) {
     BatchLayout b;
@@ -58,7 +58,8 @@ bool batch_shape_ok(const redmoe_layer* L) {
 }
 
 redmoe_status launch_batched(const redmoe_layer* L, const void* x, int T, float* out, int32_t* ids, float* w,
-                             void* ws, const redmoe_route_debug* dbg, cudaStream_t s, int* launches) {
+                             void* ws, const redmoe_route_debug* dbg, cudaStream_t s, int* launches,
+                             CacheBias cb) {
     const int H = L->hidden, E = L->n_experts, k = L->top_k, I = L->inter;
     const BatchLayout B = batch_layout(T, E, k, H, I);
     char* base = static_cast<char*>(ws);
@@ -86,7 +87,7 @@ redmoe_status launch_batched(const redmoe_layer* L, const void* x, int T, float*
     if (launches) *launches += 1;
     // 2 routing: top-k, weights, shared gate, zeroed out, grouping, tile schedule, gathered x
     if ((st = launch_route(L, x, T, logits, ids, w, sgate, counts, offsets, perm, 128, tiles, xg, bhist, ctl, s,
-                           launches)) != REDMOE_OK)
+                           launches, cb)) != REDMOE_OK)
         return st;
     if (dbg) {
         if (cudaMemcpyAsync(dbg->counts, counts, 4ull * E, cudaMemcpyDeviceToDevice, s) != cudaSuccess ||

@@ -46,6 +46,7 @@ struct RouteParams {
     int32_t* bhist;       // [grid, E]
     Control* ctl;
     uint64_t timeout_ns;
+    CacheBias cb;
 };
 
 // Exclusive prefix over v[0..n) (n <= 2 * RT_THREADS) into out[0..n); returns the total.
@@ -114,13 +115,9 @@ __global__ void __launch_bounds__(RT_THREADS, 1) route_kernel(const __grid_const
             xv[i] = c < nc ? __ldg(xr + c) : make_uint4(0u, 0u, 0u, 0u);
             gv[i] = c < nc ? __ldg(gr + c) : make_uint4(0u, 0u, 0u, 0u);
         }
-        uint32_t key[EPL];
-        const float* lr = p.logits + size_t(t) * E;
-#pragma unroll
-        for (int i = 0; i < EPL; ++i) key[i] = (i * 32 + lane < E) ? order_key(__ldcg(lr + i * 32 + lane)) : 0u;
         int id;
         float wv;
-        warp_topk_core<EPL>(key, k, id, wv);
+        warp_route<EPL>(p.logits + size_t(t) * E, E, k, p.cb.cached, p.cb.lambda, id, wv);
         if (lane < k) {
             p.ids[size_t(t) * k + lane] = id;
             p.w[size_t(t) * k + lane] = wv;
@@ -263,7 +260,7 @@ int route_smem_bytes(int E, int tpb, int k) { return 4 * (3 * E + 1 + 32 + 2 * t
 redmoe_status launch_route(const redmoe_layer* L, const void* x, int T, const float* logits, int32_t* ids, float* w,
                            float* sgate, int32_t* counts, int32_t* offsets, int32_t* perm, int tile_m,
                            int32_t* tiles, void* xg, int32_t* bhist, Control* ctl, cudaStream_t stream,
-                           int* launches) {
+                           int* launches, CacheBias cb) {
     DevInfo di;
     if (!get_dev_info(&di)) return REDMOE_ERR_CUDA;
     const int E = L->n_experts, k = L->top_k;
@@ -277,6 +274,7 @@ redmoe_status launch_route(const redmoe_layer* L, const void* x, int T, const fl
     p.ids = ids; p.w = w; p.sgate = sgate;
     p.counts = counts; p.offsets = offsets; p.perm = perm; p.tile_m = tile_m; p.tiles = tiles;
     p.xg = static_cast<uint16_t*>(xg); p.bhist = bhist; p.ctl = ctl; p.timeout_ns = BARRIER_TIMEOUT_NS;
+    p.cb = cb;
     const int smem = route_smem_bytes(E, p.tpb, k);
     if (smem > di.max_smem_optin) return REDMOE_ERR_UNSUPPORTED;
     void (*kern)(RouteParams) = E <= 256 ? route_kernel<8> : (E <= 512 ? route_kernel<16> : route_kernel<MAX_EXPERTS / 32>);

@@ -75,6 +75,61 @@ __device__ __forceinline__ void warp_topk_keys(int E, int k, const uint32_t* key
     else warp_topk_reg<MAX_EXPERTS / 32>(E, k, keys, ids, wts);
 }
 
+// Top-k of one token's E logits (global memory written earlier in the launch) by one warp,
+// optionally with the opt-in cache-aware routing bias ("Research notes, October 2026",
+// section 4: z + lambda * Delta * cached, opt-in because it changes outputs). With
+// cached != nullptr the selection ranks z[e] + lambda * Delta * cached[e], Delta the
+// token's logit range (max - min over the E logits), ties to the lower id; the weights are
+// the softmax of the unbiased logits over the selected experts (the bias changes which
+// experts run, not how their outputs are mixed). Lane j < k ends with (id_j, w_j).
+template <int EPL>
+__device__ __forceinline__ void warp_route(const float* logits, int E, int k, const uint8_t* cached, float lambda,
+                                           int& out_id, float& out_w) {
+    const int lane = threadIdx.x & 31;
+    float z[EPL];
+    uint32_t key[EPL];
+#pragma unroll
+    for (int i = 0; i < EPL; ++i) z[i] = (i * 32 + lane < E) ? __ldcg(logits + i * 32 + lane) : 0.0f;
+    if (cached == nullptr) {
+#pragma unroll
+        for (int i = 0; i < EPL; ++i) key[i] = (i * 32 + lane < E) ? order_key(z[i]) : 0u;
+        warp_topk_core<EPL>(key, k, out_id, out_w);
+        return;
+    }
+    float zmax = -INFINITY, zmin = INFINITY;
+#pragma unroll
+    for (int i = 0; i < EPL; ++i)
+        if (i * 32 + lane < E) { zmax = fmaxf(zmax, z[i]); zmin = fminf(zmin, z[i]); }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        zmax = fmaxf(zmax, __shfl_xor_sync(FULL, zmax, o));
+        zmin = fminf(zmin, __shfl_xor_sync(FULL, zmin, o));
+    }
+    const float b = lambda * (zmax - zmin);
+#pragma unroll
+    for (int i = 0; i < EPL; ++i) {
+        const int e = i * 32 + lane;
+        key[i] = e < E ? order_key(cached[e] ? z[i] + b : z[i]) : 0u;
+    }
+    float wb;
+    warp_topk_core<EPL>(key, k, out_id, wb);
+    // weights from the unbiased logits of the selection
+    const float zj = lane < k ? __ldcg(logits + out_id) : -INFINITY;
+    float m = zj;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(FULL, m, o));
+    const float ex = lane < k ? expf(zj - m) : 0.0f;
+    out_w = ex / warp_sum(ex);
+}
+
+// warp_route with EPL chosen from E.
+__device__ __forceinline__ void warp_route_any(const float* logits, int E, int k, const uint8_t* cached, float lambda,
+                                               int& out_id, float& out_w) {
+    if (E <= 256) warp_route<8>(logits, E, k, cached, lambda, out_id, out_w);
+    else if (E <= 512) warp_route<16>(logits, E, k, cached, lambda, out_id, out_w);
+    else warp_route<MAX_EXPERTS / 32>(logits, E, k, cached, lambda, out_id, out_w);
+}
+
 // Same, loading the logits (global memory written earlier) into the key buffer first.
 __device__ __forceinline__ void warp_topk(const float* logits, int E, int k, uint32_t* keys, int* ids, float* wts) {
     const int lane = threadIdx.x & 31;

@@ -52,11 +52,14 @@ def check_order(logits_row, ids):
     return bool(np.all(np.diff(l) <= GAP))
 
 
-def reference(shape, L, x_dev, gpu_ids=None, rows=None):
+def reference(shape, L, x_dev, gpu_ids=None, rows=None, cache=None):
     """Oracle routing + outputs for the device layer L and input x_dev.
 
     With gpu_ids given, exempt tokens take the oracle-enumerated set equal to the GPU's
-    (if any); returns dict with ids/w (oracle order for that set), s, out, logits, exempt.
+    (if any); returns dict with ids/w (oracle order for that set), s, out, logits (the
+    logits the selection ranks), exempt. cache = (cached mask [E], lambda) selects the
+    opt-in cache-aware routing; its near-tie rule applies to the biased logits, and the
+    weights of a matched set are renormalised from the unbiased ones.
     """
     x = mi.to_numpy(x_dev)
     lay = host_routing_layer(L)
@@ -64,10 +67,14 @@ def reference(shape, L, x_dev, gpu_ids=None, rows=None):
     T = x.shape[0]
     ids = r["ids"].copy()
     w = r["w"].copy()
+    sel_logits = r["logits"]
+    if cache is not None:
+        c = oracle.cache_route(r["logits"], np.asarray(cache[0], np.uint8), float(cache[1]), shape.k)
+        ids, w, sel_logits = c["ids"].copy(), c["w"].copy(), c["biased"]
     exempt = np.zeros(T, bool)
     bad = []
     for t in range(T):
-        sets, ex = candidate_sets(r["logits"][t], shape.k)
+        sets, ex = candidate_sets(sel_logits[t], shape.k)
         exempt[t] = ex
         if not ex or gpu_ids is None:
             continue
@@ -76,22 +83,22 @@ def reference(shape, L, x_dev, gpu_ids=None, rows=None):
             bad.append(t)
             continue
         # oracle order for the matched set: logit desc, id asc
-        chosen = sorted(g, key=lambda e: (-r["logits"][t][e], e))
+        chosen = sorted(g, key=lambda e: (-sel_logits[t][e], e))
         ids[t] = chosen
         w[t] = oracle.renorm(r["logits"][t], np.array(chosen, np.int32))
     rows = np.arange(T) if rows is None else np.asarray(rows)
     used = sorted(set(ids[rows].reshape(-1).tolist()))
     lay_e = mi.layer_to_numpy(L, experts=used)
     out = oracle.experts(lay_e, shape, x[rows], ids[rows], w[rows], r["s"][rows])
-    return dict(ids=ids, w=w, s=r["s"], out=out, logits=r["logits"], exempt=exempt, bad=bad, rows=rows)
+    return dict(ids=ids, w=w, s=r["s"], out=out, logits=sel_logits, exempt=exempt, bad=bad, rows=rows)
 
 
-def assert_layer_parity(shape, L, x_dev, out_gpu, ids_gpu, w_gpu, out_tol, w_tol, label="", rows=None):
+def assert_layer_parity(shape, L, x_dev, out_gpu, ids_gpu, w_gpu, out_tol, w_tol, label="", rows=None, cache=None):
     """rows: token rows whose outputs are checked (all by default); ids and weights are
     always checked for every token."""
     ids_g = ids_gpu.detach().cpu().numpy()
     w_g = w_gpu.detach().cpu().numpy().astype(np.float64)
-    ref = reference(shape, L, x_dev, gpu_ids=ids_g, rows=rows)
+    ref = reference(shape, L, x_dev, gpu_ids=ids_g, rows=rows, cache=cache)
     out_g = out_gpu.detach().cpu().numpy().astype(np.float64)[ref["rows"]]
     assert not ref["bad"], f"{label}: GPU top-k outside the valid near-tie sets for tokens {ref['bad']}"
     T = ids_g.shape[0]

@@ -13,6 +13,7 @@ pytestmark = pytest.mark.gpu
 
 QWEN = mi.LayerShape(H=2048, E=512, k=10, I=512, Is=512)
 QWEN_INT4 = mi.LayerShape(H=2048, E=512, k=10, I=512, Is=512, expert_dtype="int4g32")
+QWEN_INT2 = mi.LayerShape(H=2048, E=512, k=10, I=512, Is=512, expert_dtype="int2g32")
 TINY = mi.WORKLOADS["tiny_f32"]["shape"]
 
 
@@ -63,11 +64,31 @@ def test_qwen_int4(gpu_lib, T):
     assert_layer_parity(shape, L, x, out, ids, w, ot, wt, f"int4 T={T}")
 
 
-def test_repeat_calls_are_identical(gpu_lib):
+def test_qwen_int2(gpu_lib):
+    """The library's int2 group-32 experts, dequantised inside the one-row kernel."""
+    shape = QWEN_INT2
+    for seed in (6001, 6002):
+        L = _dev_layer(shape, seed)
+        x = mi.make_x(shape, 1, seed, "cuda")
+        out, ids, w, _, _ = _run(gpu_lib, shape, L, x)
+        ot, wt = tolerances(shape)
+        assert_layer_parity(shape, L, x, out, ids, w, ot, wt, f"int2 seed={seed}")
+
+
+def test_int2_beyond_one_row_is_unsupported(gpu_lib):
+    shape = QWEN_INT2
+    L = _dev_layer(shape, 6003)
+    x = mi.make_x(shape, 2, 6003, "cuda")
+    with pytest.raises(smg.RedmoeError) as e:
+        _run(gpu_lib, shape, L, x)
+    assert e.value.status == 2  # REDMOE_ERR_UNSUPPORTED
+
+
+@pytest.mark.parametrize("T,shape", [(1, QWEN), (1, QWEN_INT4), (1, QWEN_INT2), (2, QWEN)])
+def test_repeat_calls_are_identical(gpu_lib, T, shape):
     """The decode path has no atomics: two calls give bit-identical outputs."""
-    shape = QWEN
     L = _dev_layer(shape, 1234)
-    x = mi.make_x(shape, 2, 1234, "cuda")
+    x = mi.make_x(shape, T, 1234, "cuda")
     out1, ids1, w1, ws, lay = _run(gpu_lib, shape, L, x)
     out2 = torch.empty_like(out1)
     ids2 = torch.empty_like(ids1)
@@ -77,7 +98,7 @@ def test_repeat_calls_are_identical(gpu_lib):
     assert torch.equal(out1, out2) and torch.equal(ids1, ids2) and torch.equal(w1, w2)
 
 
-@pytest.mark.parametrize("T,nl,shape", [(2, 4, QWEN), (3, 3, QWEN), (1, 6, QWEN_INT4), (4, 2, TINY)])
+@pytest.mark.parametrize("T,nl,shape", [(2, 4, QWEN), (3, 3, QWEN), (1, 6, QWEN_INT4), (1, 3, QWEN), (1, 4, QWEN_INT2), (4, 2, TINY)])
 def test_stack_matches_per_layer_oracle(gpu_lib, T, nl, shape):
     layers = [_dev_layer(shape, 2000 + 17 * l) for l in range(nl)]
     xs = [mi.make_x(shape, T, 2000 + 17 * l, "cuda") for l in range(nl)]
@@ -131,11 +152,11 @@ def test_router_entry_point(gpu_lib):
 
 
 @pytest.mark.parametrize("name,T", [("bf16", 1), ("bf16", 2), ("bf16", 3), ("bf16", 4), ("int4", 1), ("int4", 3),
-                                    ("tiny", 4)])
+                                    ("int2", 1), ("tiny", 4)])
 def test_decode_after_shared_memory_poison(gpu_lib, name, T):
     """Every SM's shared memory is filled with NaN right before the call, so a read of a
     ring stage, of x or of h ahead of its data shows up in the results of this call."""
-    shape = {"bf16": QWEN, "int4": QWEN_INT4, "tiny": TINY}[name]
+    shape = {"bf16": QWEN, "int4": QWEN_INT4, "int2": QWEN_INT2, "tiny": TINY}[name]
     if name == "tiny":
         L = {k: (v.cuda() if v is not None else None) for k, v in mi.make_layer(shape, 5, "cpu").items()}
         x = mi.make_x(shape, T, 5, "cpu").cuda()

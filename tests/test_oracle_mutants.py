@@ -37,8 +37,11 @@ MUTANTS = {
     "cache_delta_is_max_only": ("const double delta = zmax - zmin;", "const double delta = zmax;"),
     "cache_bias_sign": ("zb[e] = z[e] + lambda * delta * (cached[e] ? 1.0 : 0.0);",
                         "zb[e] = z[e] - lambda * delta * (cached[e] ? 1.0 : 0.0);"),
-    "scale_group_index": ("double s = bf16_bits_to_double(scale[n * (K / 32) + c / 32]);",
-                          "double s = bf16_bits_to_double(scale[n * (K / 32) + (c / 32 + 1) % (K / 32)]);"),
+    "int2_code_order": ("int code = (byte >> (2 * (c % 4))) & 3;", "int code = (byte >> (6 - 2 * (c % 4))) & 3;"),
+    "int2_code_offset": ("return group_scale(scale, K, n, c) * (double)(code - 2);",
+                         "return group_scale(scale, K, n, c) * (double)(code - 1);"),
+    "scale_group_index": ("return bf16_bits_to_double(scale[n * (K / 32) + c / 32]);",
+                          "return bf16_bits_to_double(scale[n * (K / 32) + (c / 32 + 1) % (K / 32)]);"),
 }
 
 

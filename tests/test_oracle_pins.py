@@ -149,6 +149,61 @@ def test_int4_layer_equals_its_dequantised_fp32_copy():
     np.testing.assert_array_equal(a["out"], b["out"])
 
 
+# ----------------------------------------------------------------- int2 format
+def test_int2_hand_decoded_rows():
+    g = json.load(open(os.path.join(GOLDEN, "int2_groups.json")))
+    r0 = g["rows"][0]
+    got = oracle.dequant_int2(np.array([r0["bytes"]], np.uint8), np.array([r0["scales_bf16_bits"]], np.uint16))
+    np.testing.assert_array_equal(got[0], np.array(r0["expected"]))
+    r1 = g["rows"][1]
+    got = oracle.dequant_int2(np.array([r1["bytes"]], np.uint8), np.array([r1["scales_bf16_bits"]], np.uint16))
+    pat = r1["expected_pattern"]
+    expect = np.array([pat[0][i % 4] for i in range(32)] + [pat[1][i % 4] for i in range(32)])
+    np.testing.assert_array_equal(got[0], expect)
+
+
+def test_int2_quantiser_roundtrip_and_extremes():
+    g = torch.Generator().manual_seed(6)
+    w = torch.randn(5, 64, generator=g) * 0.02
+    w[1, 0:32] = 0.0                        # an all-zero group: scale 0, codes 2 (value 0)
+    packed, scales = mi.quantize_int2g32(w)
+    assert packed.shape == (5, 16) and scales.shape == (5, 2)
+    assert np.all(mi.to_numpy(packed)[1, 0:8] == 0xAA)
+    deq = oracle.dequant_int2(mi.to_numpy(packed), mi.to_numpy(scales))
+    s = np.repeat(scales.float().numpy().astype(np.float64), 32, axis=1)
+    # every value is -s, 0 or s, and it is the one nearest to w (scale = bf16(amax))
+    q = np.where(s == 0, 0.0, deq / np.where(s == 0, 1.0, s))
+    assert set(np.unique(q).tolist()) <= {-1.0, 0.0, 1.0}
+    wd = w.double().numpy()
+    assert np.all(np.abs(deq - wd) <= 0.5 * s * (1 + 1e-6) + np.maximum(0, np.abs(wd) - s))
+    grp = w.reshape(5, 2, 32)
+    arg = grp.abs().argmax(dim=-1)
+    for n in range(5):
+        for gi in range(2):
+            if n == 1 and gi == 0:
+                continue
+            c = gi * 32 + int(arg[n, gi])
+            assert abs(q[n, c]) == 1.0
+
+
+def test_int2_layer_equals_its_dequantised_fp32_copy():
+    shape = mi.LayerShape(H=64, E=8, k=2, I=32, Is=32, expert_dtype="int2g32", sigma=0.2)
+    lay, x = _tiny(shape, 12)
+    dq = dict(lay)
+    for w_name, s_name in (("w_gate", "s_gate"), ("w_up", "s_up"), ("w_down", "s_down")):
+        W, S = lay[w_name], lay[s_name]
+        dq[w_name] = np.stack([oracle.dequant_int2(W[e], S[e]) for e in range(W.shape[0])]).astype(np.float32)
+        dq[s_name] = None
+    for w_name, s_name in (("sh_gate", "sh_s_gate"), ("sh_up", "sh_s_up"), ("sh_down", "sh_s_down")):
+        dq[w_name] = oracle.dequant_int2(lay[w_name], lay[s_name]).astype(np.float32)
+        dq[s_name] = None
+    shape32 = mi.LayerShape(**{**shape.__dict__, "expert_dtype": "f32"})
+    a = oracle.forward(lay, shape, x)
+    b = oracle.forward(dq, shape32, x)
+    np.testing.assert_array_equal(a["ids"], b["ids"])
+    np.testing.assert_array_equal(a["out"], b["out"])
+
+
 # ------------------------------------------------------------ top-k selection
 @pytest.mark.parametrize("name", list(SHAPES))
 def test_topk_is_best_k_subset(name):
