@@ -65,6 +65,11 @@ WORKLOADS = {
                     desc="48 distinct Qwen3-Next-shaped layers, int2 group-32 experts, decode T=1"),
     "prefill": dict(shape=QWEN_ZIPF, T=2048, layers=1, stack=False, seed=3000, kernel="layer (4 kernels)",
                     desc="Qwen3-Next-shaped MoE layer, bf16, 2048-token prefill chunk, Zipf(1.1) router offsets"),
+    # one token per step through one bf16 layer whose routed experts stay in pinned host
+    # memory behind a 64-slot device cache (Zipf(1.1) router offsets make some experts hot)
+    "hostexp": dict(shape=QWEN_ZIPF, T=1, layers=1, stack=False, seed=6000, kernel="host experts (4 kernels)",
+                    desc="Qwen3-Next-shaped MoE layer, bf16, decode T=1, routed experts in pinned host memory "
+                         "behind a 64-slot device cache, Zipf(1.1) router offsets", slots=64, tokens=100),
     # the same chunk with unbiased routing: every expert is touched, so the step streams all
     # 512 experts' weights and the HBM floor moves above the tensor-core one
     "prefill_uniform": dict(shape=QWEN, T=2048, layers=1, stack=False, seed=3000, kernel="layer (4 kernels)",
@@ -412,33 +417,30 @@ def capture(step, n, stream):
 
 
 class GraphRunner:
-    """Replays n steps as whole CUDA graphs: full rotations of the layers, then one graph
-    of the remaining steps, so that no eager host call sits between timed launches."""
+    """Replays n consecutive steps (step 0 .. n-1) as whole CUDA graphs of up to CHUNK steps
+    each, so that no eager host call sits between timed launches and a timed region of up
+    to CHUNK steps is a single graph launch."""
 
-    def __init__(self, step, chunk, stream):
-        self.step, self.chunk, self.stream = step, chunk, stream
+    CHUNK = 4096
+
+    def __init__(self, step, stream):
+        self.step, self.stream = step, stream
         self.graphs = {}
 
-    def _graph(self, n):
-        if n not in self.graphs:
-            self.graphs[n] = capture(self.step, n, self.stream)
-        return self.graphs[n]
+    def _capture(self, start, n):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=self.stream):
+            for i in range(start, start + n):
+                self.step(i)
+        return g
 
-    def prepare(self, *counts):
-        for n in counts:
-            full, rem = divmod(n, self.chunk)
-            if full:
-                self._graph(self.chunk)
-            if rem:
-                self._graph(rem)
+    def prepare(self, n):
+        if n not in self.graphs:
+            self.graphs[n] = [self._capture(s, min(self.CHUNK, n - s)) for s in range(0, n, self.CHUNK)]
 
     def run(self, n):
-        full, rem = divmod(n, self.chunk)
-        g = self.graphs.get(self.chunk)
-        for _ in range(full):
+        for g in self.graphs[n]:
             g.replay()
-        if rem:
-            self.graphs[rem].replay()
 
 
 def distinct_experts(B):
@@ -458,12 +460,14 @@ def gpu_arm(args, wl, world, rank, local, B=None, name=None):
         step(0)  # one eager call: per-device set-up (attributes, driver entry points) outside capture
     torch.cuda.synchronize()
     K, W = args.steps, args.warmup
-    runner = GraphRunner(step, 1 if wl["stack"] else wl["layers"], stream)
-    runner.prepare(W, K)
+    runner = GraphRunner(step, stream)
+    runner.prepare(W)
+    runner.prepare(K)
     torch.cuda.synchronize()
 
     with torch.cuda.stream(stream):
-        runner.run(W)
+        runner.run(W)   # the W warm-up steps
+        runner.run(K)   # one untimed replay of the timed graphs (their first launch uploads them)
     torch.cuda.synchronize()
     smg.redmoe_check_timeout(B["work"], stream=stream)
 
@@ -524,7 +528,8 @@ def gpu_arm(args, wl, world, rank, local, B=None, name=None):
                          f"({wl['layers']} distinct layers)" if not wl["stack"] else
                          f"inputs larger than L2: {wl['layers']} distinct layers per step",
                    "parallelism": "replicas" if world > 1 else "single GPU",
-                   "timing": "CUDA graph replay of exactly the timed steps"},
+                   "timing": "CUDA graph replay of exactly the timed steps (one graph up to 4096 steps); "
+                             "untimed before it: the warm-up steps and one replay of the timed graph"},
         "roofline": roof,
         "e2e": e2e,
         "gpu_launches": launches,
@@ -584,6 +589,98 @@ def e2e_arm(args, wl, smg, B, stream, world):
                    "host wall clock around the K steps"}
 
 
+def host_link_gbs(nbytes=512 * 2**20, reps=5):
+    """Host-to-device copy rate from pinned memory (the link the host-expert fills use)."""
+    h = torch.empty(nbytes, dtype=torch.uint8).pin_memory()
+    d = torch.empty(nbytes, dtype=torch.uint8, device="cuda")
+    d.copy_(h, non_blocking=True)
+    torch.cuda.synchronize()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev0.record()
+    for _ in range(reps):
+        d.copy_(h, non_blocking=True)
+    ev1.record()
+    torch.cuda.synchronize()
+    return reps * nbytes / (ev0.elapsed_time(ev1) / 1e3) / 1e9
+
+
+def hostexp_arm(args, wl, world, rank, local):
+    """Decode tokens through a layer whose routed experts live in pinned host memory, served
+    by redmoe_forward_host_experts through a bounded device cache. Reports tokens/s, the
+    cache hit rate and the fill traffic against the measured host-to-device copy rate."""
+    import sparse_moe_gemv_b200 as smg
+    smg.load()
+    shape, n = wl["shape"], wl["tokens"]
+    L = mi.make_layer(shape, wl["seed"], "cuda")
+    Lh = dict(L)
+    for name in ("w_gate", "w_up", "w_down", "s_gate", "s_up", "s_down"):
+        if L.get(name) is not None:
+            Lh[name] = L[name].cpu().pin_memory()
+            L[name] = None
+    torch.cuda.empty_cache()
+    lay = smg.Layer.from_shape(Lh, shape)
+    cache = smg.ExpertCache(lay, wl["slots"])
+    ws = smg.new_workspace(lay, 1)
+    xs = [mi.make_x(shape, 1, wl["seed"] + 1 + i, "cuda") for i in range(n)]
+    out = torch.empty(1, shape.H, device="cuda")
+    ids = torch.empty(1, shape.k, dtype=torch.int32, device="cuda")
+    w = torch.empty(1, shape.k, device="cuda")
+    stream = torch.cuda.Stream()
+
+    def step(i):
+        smg.redmoe_forward_host_experts(lay, xs[i % n], out, ids, w, cache, ws, stream=stream)
+
+    K, W = args.steps, args.warmup
+    smg.redmoe_expert_cache_init(lay, cache, stream=stream)
+    with torch.cuda.stream(stream):
+        step(0)
+    torch.cuda.synchronize()
+    runner = GraphRunner(step, stream)
+    try:
+        runner.prepare(K)
+        timing = "CUDA graph replay of the timed steps"
+    except RuntimeError:  # capture refused: time eager launches instead
+        torch.cuda.synchronize()
+        runner = None
+        timing = "eager launches (graph capture refused)"
+    # warm-up: the first W tokens of the stream, then the cache starts empty again
+    with torch.cuda.stream(stream):
+        for i in range(W):
+            step(i)
+    torch.cuda.synchronize()
+    smg.redmoe_expert_cache_init(lay, cache, stream=stream)
+    torch.cuda.synchronize()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clk:
+        with torch.cuda.stream(stream):
+            ev0.record(stream)
+            if runner is not None:
+                runner.run(K)
+            else:
+                for i in range(K):
+                    step(i)
+            ev1.record(stream)
+        torch.cuda.synchronize()
+    smg.redmoe_check_timeout(ws, stream=stream)
+    el = ev0.elapsed_time(ev1) / 1e3
+    st = cache.tensors["stats"].cpu().tolist()
+    tokens, hits, misses = st[0], st[1], st[2]
+    eb = expert_bytes(shape)
+    link = host_link_gbs()
+    fill_gbs = misses * eb / el / 1e9
+    return {"workload": wl["desc"], "value": K / el, "unit": "tokens/s", "ms_per_step": el * 1e3 / K, "steps": K,
+            "warmup": W, "dtype": shape.expert_dtype,
+            "cache": {"slots": wl["slots"], "slot_bytes": smg.redmoe_expert_cache_slot_bytes(lay),
+                      "tokens": tokens, "hits": hits, "misses": misses,
+                      "hit_rate": hits / max(1, hits + misses), "starts": "empty"},
+            "timing": timing,
+            "roofline": {"bound": "host link", "achieved": fill_gbs, "peak": link, "unit": "GB/s",
+                         "frac": fill_gbs / link, "traffic": None, "kernel": wl["kernel"],
+                         "bytes_per_step": misses * eb / K,
+                         "peak_source": "pinned host-to-device copy measured in this run"},
+            "gpu_launches": 4 * K, "clocks": clk.summary()}
+
+
 MIDBATCH_T = (1, 2, 3, 4, 5, 8, 16, 32, 64, 128, 256)
 
 
@@ -608,10 +705,10 @@ def midbatch_sweep(args, world, rank, local):
             step(0)
         torch.cuda.synchronize()
         reps = max(2, min(args.steps, 240) // nl)
-        runner = GraphRunner(step, nl, stream)
+        runner = GraphRunner(step, stream)
         runner.prepare(nl * reps)
         with torch.cuda.stream(stream):
-            runner.run(nl * 2)
+            runner.run(nl * reps)  # warm-up, and the graph's upload
         torch.cuda.synchronize()
         ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         with torch.cuda.stream(stream):
@@ -635,11 +732,14 @@ def midbatch_sweep(args, world, rank, local):
             "rows": rows}
 
 
-SUB_WORKLOADS = ("fewrow_t2", "fewrow_t3", "int4_48", "int2_48", "prefill", "prefill_uniform")
-SUB_STEPS = {"fewrow_t2": 200, "fewrow_t3": 200, "int4_48": 100, "int2_48": 100, "prefill": 50, "prefill_uniform": 30}
+SUB_WORKLOADS = ("fewrow_t2", "fewrow_t3", "int4_48", "int2_48", "prefill", "prefill_uniform", "hostexp")
+SUB_STEPS = {"fewrow_t2": 200, "fewrow_t3": 200, "int4_48": 100, "int2_48": 100, "prefill": 50, "prefill_uniform": 30,
+             "hostexp": 100}
 
 
 def sub_result(res):
+    if "cache" in res:  # hostexp reports its own object
+        return res
     keep = ("value", "unit", "ms_per_step", "steps", "warmup", "dtype", "roofline", "e2e", "gpu_launches", "clocks")
     d = {k: res[k] for k in keep}
     d["workload"] = res["config"]["workload"]
@@ -654,6 +754,32 @@ def free(B):
     torch.cuda.empty_cache()
 
 
+def run_sub_workload(args, name):
+    """One extra workload of the default line, in a child process with a CUDA context of its
+    own, so that the workloads share no device state; returns (object, cpu-baseline extras)."""
+    import subprocess
+    cmd = [sys.executable, os.path.abspath(__file__), "--workload", name, "--steps", str(min(args.steps, SUB_STEPS[name])),
+           "--warmup", "3", "--sub"]
+    if not args.no_cpu_baseline:
+        cmd.append("--sub-cpu")
+    r = subprocess.run(cmd, capture_output=True, text=True, timeout=900)
+    lines = [ln for ln in r.stdout.splitlines() if ln.startswith("{")]
+    if r.returncode != 0 or not lines:
+        tail = (r.stderr or r.stdout).strip().splitlines()[-1:] or ["no output"]
+        return {"workload": WORKLOADS[name]["desc"], "error": f"exit {r.returncode}: {tail[0][:300]}"}, {}
+    d = json.loads(lines[-1])
+    return sub_result(d), d.get("cpu_extra", {})
+
+
+def sub_cpu_extra(name, B):
+    """The oracle timings that belong to a workload (rank 0, N = 1)."""
+    if name == "fewrow_t2":
+        return {"fewrow_t2_stack": cpu_oracle_stack(WORKLOADS[name], B, T=2)}
+    if name == "prefill":
+        return {"prefill_chunk": cpu_oracle_prefill(WORKLOADS[name], B)}
+    return {}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -666,6 +792,8 @@ def main():
                     help="default run: skip the objects of the other workloads")
     ap.add_argument("--layers", type=int, default=None,
                     help="override the number of distinct layers (small cases for profiler captures)")
+    ap.add_argument("--sub", action="store_true", help=argparse.SUPPRESS)      # child of the default line
+    ap.add_argument("--sub-cpu", action="store_true", help=argparse.SUPPRESS)  # child also times its oracle leg
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
@@ -687,33 +815,28 @@ def main():
         if world > 1:
             torch.distributed.destroy_process_group()
         return
+    if args.workload == "hostexp":
+        res = hostexp_arm(args, wl, world, rank, local)
+        if rank == 0:
+            print(json.dumps(res), flush=True)
+        return
+    if args.sub:
+        res, B = gpu_arm(args, wl, world, rank, local, name=args.workload)
+        if args.sub_cpu:
+            res["cpu_extra"] = sub_cpu_extra(args.workload, B)
+        print(json.dumps(res), flush=True)
+        return
     cpu = world == 1 and rank == 0 and not args.no_cpu_baseline
     res, B = gpu_arm(args, wl, world, rank, local)
     free(B)
     extra_cpu = {}
-    if args.workload == "decode_t1" and not args.no_extra:
-        fewrow_B = None
+    if args.workload == "decode_t1" and not args.no_extra and world == 1:
+        # the other workloads, each in a process of its own (one GPU: at N > 1 the line
+        # carries the headline workload only)
         for name in SUB_WORKLOADS:
-            swl = WORKLOADS[name]
-            sargs = argparse.Namespace(**{**vars(args), "steps": min(args.steps, SUB_STEPS[name]), "warmup": 3,
-                                          "workload": name})
-            reuse = None
-            if name == "fewrow_t3" and fewrow_B is not None:
-                import sparse_moe_gemv_b200 as smg
-                reuse = build_workload(swl, smg, tens=fewrow_B["tens"])  # same 12 layers, T=3 buffers
-                free(fewrow_B)
-            sub, Bs = gpu_arm(sargs, swl, world, rank, local, B=reuse, name=name)
-            res[name] = sub_result(sub)
-            if cpu and name == "fewrow_t2":
-                extra_cpu["fewrow_t2_stack"] = cpu_oracle_stack(swl, Bs, T=2)
-            if cpu and name == "prefill":
-                extra_cpu["prefill_chunk"] = cpu_oracle_prefill(swl, Bs)
-            if name == "fewrow_t2":
-                fewrow_B = Bs  # the T=3 stack runs on the same 12 layers
-            else:
-                free(Bs)
-                if name == "fewrow_t3":
-                    fewrow_B = None
+            obj, cpu_extra = run_sub_workload(args, name)
+            res[name] = obj
+            extra_cpu.update(cpu_extra)
     if rank == 0:
         if cpu:
             res["cpu_baseline"] = cpu_oracle_sample(wl)

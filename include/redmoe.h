@@ -163,6 +163,64 @@ redmoe_status redmoe_forward_cached(const redmoe_layer *L, const void *x, int32_
                                     int32_t *topk_ids, float *topk_w, const uint8_t *cached, float lambda,
                                     void *workspace, size_t workspace_bytes, void *stream);
 
+/* ---------------------------------------------------------------------------------
+ * Routed experts in host memory, served through a bounded device cache.
+ *
+ * The pages keep the dense and shared weights resident and stream routed experts into a
+ * bounded expert cache whose per-expert hotness is halved every 16 tokens ("Research
+ * notes, October 2026", section 1, SSD streaming bullets), with router-driven prefetch for
+ * the next MoE layer ("Architecture", "Future native Red Metal path"). Here the slow tier
+ * is pinned host memory that the GPU reads over the host link, and the cache is a set of
+ * device slots. All arrays below are caller-owned DEVICE memory, 16-byte aligned. */
+typedef struct redmoe_expert_cache {
+    int32_t n_slots;          /* S: slots, at least top_k                                     */
+    void *slot_gate;          /* [S, I, H] in the layer's expert dtype (int4/int2: packed)     */
+    void *slot_up;            /* [S, I, H]                                                     */
+    void *slot_down;          /* [S, H, I]                                                     */
+    void *slot_s_gate;        /* int4/int2: bf16 [S, I, H/32] scales; bf16 experts: NULL       */
+    void *slot_s_up;          /* int4/int2: bf16 [S, I, H/32]                                  */
+    void *slot_s_down;        /* int4/int2: bf16 [S, H, I/32]                                  */
+    int32_t *slot_of;         /* [E]: slot holding expert e, or -1                             */
+    int32_t *expert_in;       /* [S]: expert held by slot s, or -1                             */
+    float *hot;               /* [E]: hotness, +1 per routed token, halved every 16 tokens     */
+    int32_t *stats;           /* [4]: tokens, hits, misses (filled by calls), prefetch fills   */
+    int32_t *fill;            /* [257]: the last call's fill list (count, then expert/slot)    */
+} redmoe_expert_cache;
+
+/* Bytes of one cache slot for this layer: one routed expert's three matrices, with int4 /
+ * int2 scales (0 if the layer is invalid). slot_* arrays hold n_slots such experts. */
+size_t redmoe_expert_cache_slot_bytes(const redmoe_layer *L);
+
+/* Empty the cache on `stream`: every slot free, hotness and counters zero. */
+redmoe_status redmoe_expert_cache_init(const redmoe_layer *L, redmoe_expert_cache *cache, void *stream);
+
+/* redmoe_forward for one token row (T = 1) whose routed expert stacks (w_gate, w_up,
+ * w_down and their scales) may live in pinned host memory that the device can read
+ * (cudaHostAlloc / cudaHostRegister, e.g. torch pin_memory); router, shared gate and
+ * shared expert stay in device memory. Four launches on `stream`, no host round trip:
+ * the router; a one-block directory update (hotness += 1 for each selected expert and
+ * halved when the token count crosses a multiple of 16; each selected expert that is not
+ * resident takes a free slot, else the slot of the resident expert with the lowest
+ * hotness that this call does not use, ties to the lower slot); the copy of the missing
+ * experts from host memory into their slots; the one-row decode kernel reading expert e
+ * from slot slot_of[e] with the router's selection. The result is the layer's result
+ * (the cache changes where weights are read from, never the arithmetic). Needs the
+ * one-row kernel's layers (bf16 x/router; bf16, int4 or int2 experts; hidden <= 2048,
+ * intermediate 512; top_k <= 11, n_experts <= 512): REDMOE_ERR_UNSUPPORTED otherwise or
+ * for T != 1. REDMOE_ERR_INVALID_ARG if a routed stack is memory the device cannot read,
+ * or the cache is malformed. Workspace: redmoe_workspace_bytes(L, 1). */
+redmoe_status redmoe_forward_host_experts(const redmoe_layer *L, const void *x, int32_t T, float *out,
+                                          int32_t *topk_ids, float *topk_w, redmoe_expert_cache *cache,
+                                          void *workspace, size_t workspace_bytes, void *stream);
+
+/* Router-driven prefetch: bring the n experts `ids` (device int32, 0 <= n <= 128, each in
+ * [0, E)) into the cache on `stream` without counting them as used (no hotness, no
+ * token), e.g. the experts the next layer's router picks from the current hidden state,
+ * on a second stream while this layer computes. Victims are chosen as above; experts
+ * already resident stay. Workspace: at least the 256-byte control block. */
+redmoe_status redmoe_expert_cache_prefetch(const redmoe_layer *L, redmoe_expert_cache *cache, const int32_t *ids,
+                                           int32_t n, void *workspace, size_t workspace_bytes, void *stream);
+
 /* The router stage alone: logits, top-k ids, renormalised weights, shared gate.
  *   topk_ids [T, k] int32, topk_w [T, k] fp32, shared_gate [T] fp32 = sigmoid(x . g),
  *   logits [T, E] fp32 (router_bias included) or NULL. */
@@ -216,7 +274,9 @@ redmoe_status redmoe_forward_noalloc(const redmoe_layer *L, const void *x, int32
 
 /* Synchronise `stream`, then read the workspace's error word: REDMOE_ERR_TIMEOUT if an
  * in-kernel grid barrier gave up waiting (bounded at about one second) since the last
- * redmoe_workspace_init, else REDMOE_OK. REDMOE_ERR_CUDA if the stream reports an error.
+ * redmoe_workspace_init; REDMOE_ERR_INVALID_ARG if a kernel found device state it cannot
+ * use (an expert cache without a slot for a selected expert, an id out of range); else
+ * REDMOE_OK. REDMOE_ERR_CUDA if the stream reports an error.
  * workspace == NULL reads the error word of the current device's allocation-free
  * scratch (redmoe_forward_noalloc). */
 redmoe_status redmoe_check_timeout(const void *workspace, void *stream);

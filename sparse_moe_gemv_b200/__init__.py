@@ -7,8 +7,9 @@ and has no fallback: if the library is missing it raises.
 Names match the C entry points (redmoe_forward, redmoe_router, redmoe_route_build,
 redmoe_forward_stack, redmoe_forward_noalloc, redmoe_workspace_bytes,
 redmoe_workspace_init, redmoe_check_timeout, redmoe_selftest_wait_limit,
-redmoe_fill_shared_memory, redmoe_forward_cached, redmoe_status_string,
-redmoe_abi_version).
+redmoe_fill_shared_memory, redmoe_forward_cached, redmoe_expert_cache_slot_bytes,
+redmoe_expert_cache_init, redmoe_forward_host_experts, redmoe_expert_cache_prefetch,
+redmoe_status_string, redmoe_abi_version).
 """
 
 from __future__ import annotations
@@ -30,7 +31,8 @@ STATUS = {0: "REDMOE_OK", 1: "REDMOE_ERR_INVALID_ARG", 2: "REDMOE_ERR_UNSUPPORTE
 SYMBOLS = ("redmoe_abi_version", "redmoe_status_string", "redmoe_workspace_bytes", "redmoe_workspace_init",
            "redmoe_forward", "redmoe_router", "redmoe_route_build", "redmoe_forward_stack",
            "redmoe_check_timeout", "redmoe_forward_noalloc", "redmoe_selftest_wait_limit",
-           "redmoe_fill_shared_memory", "redmoe_forward_cached")
+           "redmoe_fill_shared_memory", "redmoe_forward_cached", "redmoe_expert_cache_slot_bytes",
+           "redmoe_expert_cache_init", "redmoe_forward_host_experts", "redmoe_expert_cache_prefetch")
 
 _lock = threading.Lock()
 _lib = None
@@ -53,6 +55,13 @@ class _Layer(C.Structure):
         ("sh_gate", C.c_void_p), ("sh_up", C.c_void_p), ("sh_down", C.c_void_p),
         ("sh_s_gate", C.c_void_p), ("sh_s_up", C.c_void_p), ("sh_s_down", C.c_void_p),
     ]
+
+
+class _ExpertCache(C.Structure):
+    _fields_ = [("n_slots", C.c_int32), ("slot_gate", C.c_void_p), ("slot_up", C.c_void_p), ("slot_down", C.c_void_p),
+                ("slot_s_gate", C.c_void_p), ("slot_s_up", C.c_void_p), ("slot_s_down", C.c_void_p),
+                ("slot_of", C.c_void_p), ("expert_in", C.c_void_p), ("hot", C.c_void_p), ("stats", C.c_void_p),
+                ("fill", C.c_void_p)]
 
 
 class _RouteDebug(C.Structure):
@@ -93,6 +102,14 @@ def load():
         lib.redmoe_selftest_wait_limit.argtypes = [P, sz, i32, C.c_uint64, P]
         lib.redmoe_forward_cached.restype = i32
         lib.redmoe_forward_cached.argtypes = [P, P, i32, P, P, P, P, C.c_float, P, sz, P]
+        lib.redmoe_expert_cache_slot_bytes.restype = sz
+        lib.redmoe_expert_cache_slot_bytes.argtypes = [P]
+        lib.redmoe_expert_cache_init.restype = i32
+        lib.redmoe_expert_cache_init.argtypes = [P, P, P]
+        lib.redmoe_forward_host_experts.restype = i32
+        lib.redmoe_forward_host_experts.argtypes = [P, P, i32, P, P, P, P, P, sz, P]
+        lib.redmoe_expert_cache_prefetch.restype = i32
+        lib.redmoe_expert_cache_prefetch.argtypes = [P, P, P, i32, P, sz, P]
         lib.redmoe_fill_shared_memory.restype = i32
         lib.redmoe_fill_shared_memory.argtypes = [C.c_uint32, P]
         if lib.redmoe_abi_version() != ABI_VERSION:
@@ -273,3 +290,63 @@ NAN_PATTERN = 0x7FC00000
 def redmoe_fill_shared_memory(pattern: int = NAN_PATTERN, stream=None) -> None:
     """Fill every SM's shared memory with a 32-bit pattern before the next launch."""
     _check(load().redmoe_fill_shared_memory(int(pattern) & 0xFFFFFFFF, _stream(stream)), "redmoe_fill_shared_memory")
+
+
+class ExpertCache:
+    """A bounded device cache of routed experts (redmoe_expert_cache): n_slots slots in the
+    layer's expert dtype plus the directory; device tensors owned by this object."""
+
+    def __init__(self, layer: "Layer", n_slots: int, device=None):
+        dev = device or "cuda"
+        H, I, E = layer.hidden, layer.inter, layer.n_experts
+        dt = layer.expert_dtype
+        per = {"bf16": 2.0, "f32": 4.0, "int4g32": 0.5, "int2g32": 0.25}[dt]
+
+        def stack(n, k):
+            return torch.empty(n_slots, int(n * k * per), dtype=torch.uint8, device=dev)
+
+        t = {"slot_gate": stack(I, H), "slot_up": stack(I, H), "slot_down": stack(H, I)}
+        if dt in ("int4g32", "int2g32"):
+            t.update(slot_s_gate=torch.empty(n_slots, I * H // 32, dtype=torch.bfloat16, device=dev),
+                     slot_s_up=torch.empty(n_slots, I * H // 32, dtype=torch.bfloat16, device=dev),
+                     slot_s_down=torch.empty(n_slots, H * I // 32, dtype=torch.bfloat16, device=dev))
+        t.update(slot_of=torch.empty(E, dtype=torch.int32, device=dev),
+                 expert_in=torch.empty(n_slots, dtype=torch.int32, device=dev),
+                 hot=torch.empty(E, dtype=torch.float32, device=dev),
+                 stats=torch.empty(4, dtype=torch.int32, device=dev),
+                 fill=torch.empty(257, dtype=torch.int32, device=dev))
+        self.tensors = t
+        st = _ExpertCache()
+        st.n_slots = n_slots
+        for name, _ in _ExpertCache._fields_[1:]:
+            setattr(st, name, _ptr(t.get(name)))
+        self.struct = st
+        self.n_slots = n_slots
+
+    @property
+    def ref(self):
+        return C.byref(self.struct)
+
+
+def redmoe_expert_cache_slot_bytes(layer: Layer) -> int:
+    return int(load().redmoe_expert_cache_slot_bytes(layer.ref))
+
+
+def redmoe_expert_cache_init(layer: Layer, cache: ExpertCache, stream=None) -> None:
+    _check(load().redmoe_expert_cache_init(layer.ref, cache.ref, _stream(stream)), "redmoe_expert_cache_init")
+
+
+def redmoe_forward_host_experts(layer: Layer, x: torch.Tensor, out: torch.Tensor, topk_ids: torch.Tensor,
+                                topk_w: torch.Tensor, cache: ExpertCache, workspace: torch.Tensor, stream=None) -> None:
+    """One token through a layer whose routed experts may be in pinned host memory."""
+    st = load().redmoe_forward_host_experts(layer.ref, _ptr(x), int(x.shape[0]), _ptr(out), _ptr(topk_ids),
+                                            _ptr(topk_w), cache.ref, _ptr(workspace),
+                                            workspace.numel() * workspace.element_size(), _stream(stream))
+    _check(st, "redmoe_forward_host_experts")
+
+
+def redmoe_expert_cache_prefetch(layer: Layer, cache: ExpertCache, ids: torch.Tensor, workspace: torch.Tensor,
+                                 stream=None) -> None:
+    st = load().redmoe_expert_cache_prefetch(layer.ref, cache.ref, _ptr(ids), int(ids.numel()), _ptr(workspace),
+                                             workspace.numel() * workspace.element_size(), _stream(stream))
+    _check(st, "redmoe_expert_cache_prefetch")

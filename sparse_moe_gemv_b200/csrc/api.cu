@@ -131,6 +131,9 @@ DecLayer dec_layer(const redmoe_layer* L, const void* x, float* out, int32_t* id
     d.out = out;
     d.ids = ids;
     d.w = w;
+    d.given_ids = nullptr;
+    d.given_w = nullptr;
+    d.slot_of = nullptr;
     return d;
 }
 
@@ -295,7 +298,8 @@ redmoe_status redmoe_check_timeout(const void* workspace, void* stream) {
     if (cudaStreamSynchronize(s) != cudaSuccess) return REDMOE_ERR_CUDA;
     Control c;
     if (cudaMemcpy(&c, workspace, sizeof(c), cudaMemcpyDeviceToHost) != cudaSuccess) return REDMOE_ERR_CUDA;
-    return (c.err & ERRBIT_TIMEOUT) ? REDMOE_ERR_TIMEOUT : REDMOE_OK;
+    if (c.err & ERRBIT_TIMEOUT) return REDMOE_ERR_TIMEOUT;
+    return (c.err & ERRBIT_STATE) ? REDMOE_ERR_INVALID_ARG : REDMOE_OK;
 }
 
 }  // extern "C"

@@ -9,7 +9,7 @@ namespace redmoe {
 enum : int { DT_F32 = 0, DT_BF16 = 1, DT_INT4 = 2, DT_INT2 = 3 };
 
 // Bits of the workspace error word.
-enum : int { ERRBIT_TIMEOUT = 1 };
+enum : int { ERRBIT_TIMEOUT = 1, ERRBIT_STATE = 2 };
 
 constexpr unsigned FULL = 0xffffffffu;
 
@@ -43,13 +43,6 @@ __device__ __forceinline__ uint32_t order_key(float f) {
 __device__ __forceinline__ float key_to_float(uint32_t k) {
     uint32_t u = (k & 0x80000000u) ? (k & 0x7fffffffu) : ~k;
     return __uint_as_float(u);
-}
-
-// int2 codes n and n+1 of w as floats (code - 2): exponent-trick conversion, exact.
-__device__ __forceinline__ float2 crumb2(uint32_t w, int n) {
-    const float a = __uint_as_float(0x4B000000u | ((w >> (2 * n)) & 3u));
-    const float b = __uint_as_float(0x4B000000u | ((w >> (2 * n + 2)) & 3u));
-    return __fadd2_rn(make_float2(a, b), make_float2(-8388610.0f, -8388610.0f));
 }
 
 // ------------------------------------------------------------------- loads

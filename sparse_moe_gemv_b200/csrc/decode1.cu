@@ -9,21 +9,22 @@
 //   * Every lane keeps its slice of x in registers as fp32 for the whole layer, so a weight
 //     chunk is dotted straight out of the registers it was loaded into: no shared-memory
 //     traffic for activations or for gate/up weights.
-//   * Phase A: warps stream the router rows, the shared-gate row and the shared expert's
-//     gate/up rows (the shared expert needs no routing: the "extra slot" of the DwarfStar
-//     MoE kernel, "Research notes, October 2026", section 1) with 16-byte vector loads.
-//     Meanwhile one thread per block starts a bulk copy of the block's rows of the shared
-//     expert's down matrix into shared memory.
-//   * Grid barrier; every warp then computes the top-k of the 512 logits in registers
-//     (router, top-k and shared gate form one stage, as in the same section). One thread
-//     per block immediately starts bulk copies of the block's rows of the k routed
-//     experts' down matrices: all of phase C's weights stream into shared memory while
-//     phase B runs, since they do not depend on h.
-//   * Phase B: each block takes an equal contiguous share of the k * I routed gate/up row
-//     pairs; each warp keeps G pairs of loads in flight and writes h = silu(a) * u.
-//   * Grid barrier; phase C computes the block's output rows from the down rows already
-//     in shared memory and h (read from L2 into registers). Each output row is summed over
-//     the experts in a fixed order: the result is deterministic.
+//   * Phase A: warps stream the router rows and the shared-gate row with 16-byte vector
+//     loads. Meanwhile one thread per block starts a bulk copy of the block's rows of the
+//     shared expert's down matrix into shared memory.
+//   * Grid barrier; one warp per block computes the top-k of the 512 logits in registers
+//     (router, top-k and shared gate form one stage: "Research notes, October 2026",
+//     section 1) while the other warps stream the shared expert's gate/up rows (the
+//     shared expert needs no routing: the "extra slot" of the DwarfStar MoE kernel, same
+//     section). Then one thread per block starts bulk copies of the block's rows of the k
+//     routed experts' down matrices: phase C's weights stream into shared memory during
+//     phase B, since they do not depend on h.
+//   * Phase B: the k * I routed gate/up row pairs, interleaved over all warps; bf16 warps
+//     keep two pairs of loads in flight, int4/int2 warps issue all of theirs at once;
+//     h = silu(a) * u.
+//   * Grid barrier; h is bulk-copied into shared memory and phase C computes the block's
+//     output rows from the down rows already there. Each output row is summed over the
+//     experts in a fixed order: the result is deterministic.
 //
 // Down rows are only I = 512 elements long (1 KiB bf16, 256 B + 32 B int4): the block's
 // rows of one expert form one contiguous range, copied in one piece, which is the lesson
@@ -45,9 +46,11 @@ constexpr int D1_THREADS = 256;
 constexpr int D1_WARPS = D1_THREADS / 32;
 constexpr int D1_XPL = 64;        // x elements per lane (H = 2048 at most)
 constexpr int D1_HPL = 16;        // h elements per lane (I = 512)
-constexpr int D1_MAXK = 16;       // routed experts per token (plus the shared one)
+constexpr int D1_MAXK = 11;       // routed experts per token (plus the shared one)
+constexpr int D1_MAXE = 512;      // experts (16 router logits per lane in the top-k)
 constexpr int D1_RB_MAX = 16;     // output rows per block
 constexpr int D1_G = 2;           // routed gate/up row pairs in flight per warp (bf16)
+constexpr int D1_GQ = 5;          // the same for int4 / int2 (all of a warp's pairs at Qwen3-Next size)
 
 __host__ __device__ constexpr int a16(int x) { return (x + 15) & ~15; }
 
@@ -110,6 +113,38 @@ __device__ __forceinline__ float2 dot_row_bf(const RowBF& r, const float (&xf)[D
     return fadd2(a, b);
 }
 
+// Packed codes to fp32 with one byte permute per element: a code c in the low bits of
+// byte b of `v` (the other bits zero) becomes the float 2^23 + c (bytes {c, 0, 0, 0x4B});
+// subtracting 2^23 + bias then gives c - bias exactly.
+__device__ __forceinline__ float code_f(uint32_t v, uint32_t b) {
+    return __uint_as_float(__byte_perm(v, 0x4B000000u, 0x7650u | b));
+}
+
+// 8 int4 elements (one word: element n in bits 4n .. 4n+3) dotted with xv[0..8)
+__device__ __forceinline__ float2 dot8_q4(uint32_t w, const float* xv, float2 a) {
+    const uint32_t lo = w & 0x0F0F0F0Fu;         // elements 0, 2, 4, 6 in bytes 0..3
+    const uint32_t hi = (w >> 4) & 0x0F0F0F0Fu;  // elements 1, 3, 5, 7
+    const float2 off = make_float2(-8388616.0f, -8388616.0f);  // -(2^23 + 8)
+#pragma unroll
+    for (uint32_t b = 0; b < 4; ++b)
+        a = ffma2(fadd2(make_float2(code_f(lo, b), code_f(hi, b)), off), make_float2(xv[2 * b], xv[2 * b + 1]), a);
+    return a;
+}
+
+// 16 int2 elements (one word: element n in bits 2n, 2n+1) dotted with xv[0..16)
+__device__ __forceinline__ float2 dot16_q2(uint32_t w, const float* xv) {
+    const uint32_t c0 = w & 0x03030303u, c1 = (w >> 2) & 0x03030303u;  // elements 4b, 4b+1
+    const uint32_t c2 = (w >> 4) & 0x03030303u, c3 = (w >> 6) & 0x03030303u;  // 4b+2, 4b+3
+    const float2 off = make_float2(-8388610.0f, -8388610.0f);  // -(2^23 + 2)
+    float2 a = make_float2(0.f, 0.f), b2 = make_float2(0.f, 0.f);
+#pragma unroll
+    for (uint32_t b = 0; b < 4; ++b) {
+        a = ffma2(fadd2(make_float2(code_f(c0, b), code_f(c1, b)), off), make_float2(xv[4 * b], xv[4 * b + 1]), a);
+        b2 = ffma2(fadd2(make_float2(code_f(c2, b), code_f(c3, b)), off), make_float2(xv[4 * b + 2], xv[4 * b + 3]), b2);
+    }
+    return fadd2(a, b2);
+}
+
 // One int4 group-32 row of H elements, in the int4 chunk layout: H / 1024 chunks of 32
 // elements (16 bytes, one scale group) per lane.
 struct RowQ4 {
@@ -132,14 +167,10 @@ __device__ __forceinline__ float2 dot_row_q4(const RowQ4& r, const float (&xf)[D
     for (int j = 0; j < D1_XPL / 32; ++j) {
         const uint32_t w[4] = {r.w[j].x, r.w[j].y, r.w[j].z, r.w[j].w};
         float2 a = make_float2(0.f, 0.f), b = make_float2(0.f, 0.f);
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-            const float* xv = xf + 32 * j + 8 * q;
-            a = ffma2(nib2(w[q], 0), make_float2(xv[0], xv[1]), a);
-            b = ffma2(nib2(w[q], 2), make_float2(xv[2], xv[3]), b);
-            a = ffma2(nib2(w[q], 4), make_float2(xv[4], xv[5]), a);
-            b = ffma2(nib2(w[q], 6), make_float2(xv[6], xv[7]), b);
-        }
+        a = dot8_q4(w[0], xf + 32 * j, a);
+        b = dot8_q4(w[1], xf + 32 * j + 8, b);
+        a = dot8_q4(w[2], xf + 32 * j + 16, a);
+        b = dot8_q4(w[3], xf + 32 * j + 24, b);
         const float s = bf16f(r.s[j]);
         acc = ffma2(make_float2(s, s), fadd2(a, b), acc);
     }
@@ -161,16 +192,6 @@ __device__ __forceinline__ void ld_row_q2(RowQ2& r, const void* row, const uint1
         r.w[j] = ok ? ld_stream(p + c) : make_uint4(0u, 0u, 0u, 0u);
         r.s[j] = ok ? ld_stream_u32(sc + 2 * c) : 0u;
     }
-}
-// 16 consecutive int2 elements (one word) dotted with xv[0..16)
-__device__ __forceinline__ float2 dot16_q2(uint32_t w, const float* xv) {
-    float2 a = make_float2(0.f, 0.f), b = make_float2(0.f, 0.f);
-#pragma unroll
-    for (int n = 0; n < 16; n += 4) {
-        a = ffma2(crumb2(w, n), make_float2(xv[n], xv[n + 1]), a);
-        b = ffma2(crumb2(w, n + 2), make_float2(xv[n + 2], xv[n + 3]), b);
-    }
-    return fadd2(a, b);
 }
 __device__ __forceinline__ float2 dot_row_q2(const RowQ2& r, const float (&xf)[D1_XPL]) {
     float2 acc = make_float2(0.f, 0.f);
@@ -215,7 +236,7 @@ __device__ __forceinline__ float hsum2(float2 v) { return warp_sum(v.x + v.y); }
 // down matrix of k + 1 experts (routed slots 0..k-1 in selection order, the shared
 // expert in slot k), each slot RB rows (int4: codes, then scales).
 struct D1Smem {
-    int dreg, slot, sc_off, bars, part, total;
+    int dreg, slot, sc_off, hbuf, bars, part, sel, total;
 };
 __host__ __device__ inline D1Smem d1_smem(int wt, int k, int I, int RB) {
     D1Smem s;
@@ -224,8 +245,10 @@ __host__ __device__ inline D1Smem d1_smem(int wt, int k, int I, int RB) {
     s.slot = a16(s.sc_off + RB * d1_scale_bytes(wt, I));
     int o = 0;
     s.dreg = o; o += (k + 1) * s.slot;
-    s.bars = o; o += 8 * (D1_MAXK + 1);
+    s.hbuf = o; o += a16(4 * k * I);  // the routed h rows, staged for phase C
+    s.bars = o; o += 8 * (D1_MAXK + 2);
     s.part = o; o += 4 * D1_WARPS * D1_RB_MAX;
+    s.sel = o; o += 12 * D1_MAXK;  // the block's top-k: ids, weights, stack indices
     s.total = a16(o);
     return s;
 }
@@ -256,7 +279,12 @@ __global__ void __launch_bounds__(D1_THREADS, 1) decode1_kernel(const __grid_con
     const D1Smem S = d1_smem(WT, k, I, RB);
     unsigned char* dreg = smem + S.dreg;
     uint64_t* dbar = reinterpret_cast<uint64_t*>(smem + S.bars);
+    uint64_t* hbar = dbar + D1_MAXK + 1;
+    const float* hbuf = reinterpret_cast<const float*>(smem + S.hbuf);
     float* part = reinterpret_cast<float*>(smem + S.part);
+    int* s_sel_id = reinterpret_cast<int*>(smem + S.sel);
+    float* s_sel_w = reinterpret_cast<float*>(smem + S.sel) + D1_MAXK;
+    int* s_sel_slot = reinterpret_cast<int*>(smem + S.sel) + 2 * D1_MAXK;
     constexpr bool PACKED = WT != DT_BF16;           // int4 / int2: codes plus group scales
     const int drow = d1_row_bytes(WT, I);            // bytes of one down row (codes)
     const int dsc = d1_scale_bytes(WT, I);           // bytes of its scales
@@ -267,6 +295,7 @@ __global__ void __launch_bounds__(D1_THREADS, 1) decode1_kernel(const __grid_con
 
     if (threadIdx.x == 0) {
         for (int i = 0; i <= k; ++i) mbar_init(dbar + i, 1);
+        mbar_init(hbar, 1);
         fence_mbar_init();
     }
     __syncthreads();
@@ -292,123 +321,50 @@ __global__ void __launch_bounds__(D1_THREADS, 1) decode1_kernel(const __grid_con
             fence_proxy_async_smem();  // the previous layer's reads of dreg come first
             issue_down(k, Ly.sh_down, Ly.sh_s_down);
         }
-        // job q < E: router row q; q == E: shared-gate row; q > E: shared gate/up row q-E-1.
-        // Warp w of block b takes q = w * nblocks + b (+ Wtot ...): every block gets a few
-        // of each kind.
-        const int jobsA = E + 1 + I;
-        for (int q = warp * nblocks + blockIdx.x; q < jobsA; q += Wtot) {
+        // job q < E: router row q; q == E: shared-gate row; q > E: the shared expert's
+        // gate/up row q - E - 1 (it needs no routing: the extra expert slot of the DwarfStar
+        // MoE kernel). Warp w of block b takes q = w * nblocks + b (+ Wtot ...): the router
+        // rows go to the low warps of every block, the shared rows to the others.
+        for (int q = warp * nblocks + blockIdx.x; q < E + 1 + I; q += Wtot) {
+            if (Ly.given_ids && q < E) continue;  // routing given: no router rows
+            float xr[D1_XPL];
             if (q <= E) {
-                float xf[D1_XPL];
                 RowBF r;
                 const void* row = q < E ? static_cast<const void*>(static_cast<const char*>(Ly.router_w) + size_t(q) * 2 * H)
                                         : Ly.shared_gate_w;
                 ld_row_bf(r, row, H, lane);
-                load_x<DT_BF16>(x, H, lane, xf);
-                const float v = hsum2(dot_row_bf(r, xf));
+                load_x<DT_BF16>(x, H, lane, xr);
+                const float v = hsum2(dot_row_bf(r, xr));
                 if (lane == 0) {
                     if (q < E) p.logits[q] = v + (Ly.router_bias ? Ly.router_bias[q] : 0.0f);
                     else *sgate = 1.0f / (1.0f + expf(-v));
                 }
             } else {
                 const int i = q - E - 1;
-                float xf[D1_XPL];
                 Row g, u;
                 ld_row<WT>(g, static_cast<const char*>(Ly.sh_gate) + size_t(i) * grow,
                            PACKED ? Ly.sh_s_gate + size_t(i) * (H / 32) : nullptr, H, lane);
                 ld_row<WT>(u, static_cast<const char*>(Ly.sh_up) + size_t(i) * grow,
                            PACKED ? Ly.sh_s_up + size_t(i) * (H / 32) : nullptr, H, lane);
-                load_x<WT>(x, H, lane, xf);
-                const float a = hsum2(dot_row<WT>(g, xf)), b = hsum2(dot_row<WT>(u, xf));
+                load_x<WT>(x, H, lane, xr);
+                const float a = hsum2(dot_row<WT>(g, xr)), b = hsum2(dot_row<WT>(u, xr));
                 if (lane == 0) hsh[i] = silu_mul(a, b);
             }
         }
         grid_barrier(p.ctl, nblocks, bar_idx++, to);
 
-        // ------------------------------------------------------------ phase B
-        // top-k of the logits by every warp, in registers: lane j < k ends with the id and
-        // the renormalised weight of selection j
-        int sel_id;
-        float sel_w;
-        if (E <= 512) warp_route<16>(p.logits, E, k, p.cb.cached, p.cb.lambda, sel_id, sel_w);
-        else warp_route<MAX_EXPERTS / 32>(p.logits, E, k, p.cb.cached, p.cb.lambda, sel_id, sel_w);
-        if (blockIdx.x == 0 && warp == 0 && lane < k) {
-            Ly.ids[lane] = sel_id;
-            Ly.w[lane] = sel_w;
-        }
-        if (warp == 0 && nrows > 0) {
-            // phase C's routed down rows do not depend on h: start their copies now
-            for (int j = 0; j < k; ++j) {
-                const int e = __shfl_sync(FULL, sel_id, j);
-                if (lane == 0)
-                    issue_down(j, static_cast<const char*>(Ly.w_down) + size_t(e) * H * drow,
-                               PACKED ? Ly.s_down + size_t(e) * H * (I / 32) : nullptr);
-            }
-        }
-        {
-            float xf[D1_XPL];
-            load_x<WT>(x, H, lane, xf);
-            // this block's share [j0, j1) of the k * I routed row pairs (u-major)
-            const int J = k * I;
-            const int j0 = int((long long)J * blockIdx.x / nblocks), j1 = int((long long)J * (blockIdx.x + 1) / nblocks);
-            constexpr int G = (WT == DT_INT2) ? 8 : ((WT == DT_INT4) ? 4 : D1_G);
-            for (int jb = j0 + warp; jb < j1; jb += D1_WARPS * G) {
-                Row g[G], u[G];
-#pragma unroll
-                for (int t = 0; t < G; ++t) {
-                    const int j = jb + t * D1_WARPS;
-                    const int uu = j / I, i = j - (j / I) * I;
-                    const int e = __shfl_sync(FULL, sel_id, uu < k ? uu : 0);
-                    if (j < j1) {
-                        const size_t rowi = size_t(e) * I + i;
-                        ld_row<WT>(g[t], static_cast<const char*>(Ly.w_gate) + rowi * grow,
-                                   PACKED ? Ly.s_gate + rowi * (H / 32) : nullptr, H, lane);
-                        ld_row<WT>(u[t], static_cast<const char*>(Ly.w_up) + rowi * grow,
-                                   PACKED ? Ly.s_up + rowi * (H / 32) : nullptr, H, lane);
-                    }
-                }
-#pragma unroll
-                for (int t = 0; t < G; ++t) {
-                    const int j = jb + t * D1_WARPS;
-                    if (j < j1) {
-                        const float a = hsum2(dot_row<WT>(g[t], xf)), b = hsum2(dot_row<WT>(u[t], xf));
-                        if (lane == 0) p.hrt[j] = silu_mul(a, b);
-                    }
-                }
-            }
-        }
-        grid_barrier(p.ctl, nblocks, bar_idx++, to);
-
-        // ------------------------------------------------------------ phase C
-        if (l + 1 < p.n_layers && threadIdx.x < 32) {
-            // L2 prefetch of the next layer's router rows and shared gate/up rows (this
-            // block's phase-A jobs of that layer)
-            const DecLayer& Nx = p.L[l + 1];
-            for (int q = lane * nblocks + blockIdx.x; q < E + 1 + I; q += 32 * nblocks) {
-                if (q < E) prefetch_l2(static_cast<const char*>(Nx.router_w) + size_t(q) * 2 * H, 2 * H);
-                else if (q > E) {
-                    prefetch_l2(static_cast<const char*>(Nx.sh_gate) + size_t(q - E - 1) * grow, grow);
-                    prefetch_l2(static_cast<const char*>(Nx.sh_up) + size_t(q - E - 1) * grow, grow);
-                }
-            }
-        }
-        // units (slot u, half hf of the block's rows): 2 (k + 1) units over the warps; each
-        // warp accumulates its rows' weighted partials in registers
+        // Phase C's work comes in units (slot u, half hf of the block's rows): the shared
+        // expert's two units (warps 1 and 2, while warp 0 takes the top-k) and the routed
+        // 2 k units (unit = warp + 8 m, every unit of a warp has hf = warp & 1). Each warp
+        // accumulates its rows' weighted partials in registers.
+        constexpr int MU = (2 * D1_MAXK + D1_WARPS - 1) / D1_WARPS;  // routed units per warp, at most
         const int half = (nrows + 1) / 2;
+        const int ra = (warp & 1) * half, rn = nrows > 0 ? min(half, nrows - ra) : 0;
         float2 acc[D1_RB_MAX / 2];
 #pragma unroll
         for (int r = 0; r < D1_RB_MAX / 2; ++r) acc[r] = make_float2(0.f, 0.f);
-        const float sg = __ldcg(sgate);
-        for (int unit = warp; nrows > 0 && unit < 2 * (k + 1); unit += D1_WARPS) {
-            const int u = unit >> 1, hf = unit & 1;
-            const int ra = hf * half, rn = min(half, nrows - ra);
-            const float* hv = (u < k ? p.hrt + size_t(u) * I : hsh) + lane * D1_HPL;
-            float hf32[D1_HPL];
-#pragma unroll
-            for (int i = 0; i < D1_HPL / 4; ++i) {
-                const float4 v = __ldcg(reinterpret_cast<const float4*>(hv) + i);
-                hf32[4 * i] = v.x; hf32[4 * i + 1] = v.y; hf32[4 * i + 2] = v.z; hf32[4 * i + 3] = v.w;
-            }
-            const float wu = u < k ? __shfl_sync(FULL, sel_w, u) : sg;
+        // weighted row dots of one unit: acc[r] += wu * (row ra + r of slot u) . h
+        auto unit_dots = [&](int u, float wu, const float (&hf32)[D1_HPL]) {
             mbar_wait(dbar + u, par, err, to);
             const unsigned char* slot = dreg + u * S.slot;
 #pragma unroll
@@ -422,42 +378,163 @@ __global__ void __launch_bounds__(D1_THREADS, 1) decode1_kernel(const __grid_con
                     } else if constexpr (WT == DT_INT4) {
                         const uint2 wv = *reinterpret_cast<const uint2*>(slot + (ra + r) * drow + lane * 8);
                         const float s = bf16f(*reinterpret_cast<const uint16_t*>(slot + S.sc_off + (ra + r) * dsc + (lane >> 1) * 2));
-                        float2 a = make_float2(0.f, 0.f);
-                        a = ffma2(nib2(wv.x, 0), make_float2(hf32[0], hf32[1]), a);
-                        a = ffma2(nib2(wv.x, 2), make_float2(hf32[2], hf32[3]), a);
-                        a = ffma2(nib2(wv.x, 4), make_float2(hf32[4], hf32[5]), a);
-                        a = ffma2(nib2(wv.x, 6), make_float2(hf32[6], hf32[7]), a);
-                        a = ffma2(nib2(wv.y, 0), make_float2(hf32[8], hf32[9]), a);
-                        a = ffma2(nib2(wv.y, 2), make_float2(hf32[10], hf32[11]), a);
-                        a = ffma2(nib2(wv.y, 4), make_float2(hf32[12], hf32[13]), a);
-                        a = ffma2(nib2(wv.y, 6), make_float2(hf32[14], hf32[15]), a);
-                        d = ffma2(make_float2(s, s), a, d);
+                        const float2 a = dot8_q4(wv.x, hf32, make_float2(0.f, 0.f));
+                        const float2 b = dot8_q4(wv.y, hf32 + 8, make_float2(0.f, 0.f));
+                        d = ffma2(make_float2(s, s), fadd2(a, b), d);
                     } else {
                         const uint4* wr = reinterpret_cast<const uint4*>(slot + (ra + r) * drow + lane * 32);
                         const uint4 w0 = wr[0], w1 = wr[1];
+                        float2 e = make_float2(0.f, 0.f);
                         d = ffma2(bf2(w0.x), make_float2(hf32[0], hf32[1]), d);
-                        d = ffma2(bf2(w0.y), make_float2(hf32[2], hf32[3]), d);
+                        e = ffma2(bf2(w0.y), make_float2(hf32[2], hf32[3]), e);
                         d = ffma2(bf2(w0.z), make_float2(hf32[4], hf32[5]), d);
-                        d = ffma2(bf2(w0.w), make_float2(hf32[6], hf32[7]), d);
+                        e = ffma2(bf2(w0.w), make_float2(hf32[6], hf32[7]), e);
                         d = ffma2(bf2(w1.x), make_float2(hf32[8], hf32[9]), d);
-                        d = ffma2(bf2(w1.y), make_float2(hf32[10], hf32[11]), d);
+                        e = ffma2(bf2(w1.y), make_float2(hf32[10], hf32[11]), e);
                         d = ffma2(bf2(w1.z), make_float2(hf32[12], hf32[13]), d);
-                        d = ffma2(bf2(w1.w), make_float2(hf32[14], hf32[15]), d);
+                        e = ffma2(bf2(w1.w), make_float2(hf32[14], hf32[15]), e);
+                        d = fadd2(d, e);
                     }
                     acc[r] = ffma2(make_float2(wu, wu), d, acc[r]);
                 }
             }
-            // a warp's units all share its half: unit = warp + 8 m keeps hf = warp & 1
+        };
+        // ------------------------------------------------------------ phase B
+        // x in the layout of the expert weights
+        float xf[D1_XPL];
+        load_x<WT>(x, H, lane, xf);
+        if (warp == 0) {
+            // one warp per block takes the top-k of the logits (lane j < k: id and
+            // renormalised weight of selection j) and shares it
+            int id = 0;
+            float wv = 0.0f;
+            if (Ly.given_ids) {
+                if (lane < k) {
+                    id = __ldcg(Ly.given_ids + lane);
+                    wv = __ldcg(Ly.given_w + lane);
+                }
+            } else {
+                warp_route<D1_MAXE / 32>(p.logits, E, k, p.cb.cached, p.cb.lambda, id, wv);
+            }
+            if (lane < k) {
+                int slot = id;
+                if (Ly.slot_of) {
+                    slot = __ldcg(Ly.slot_of + id);
+                    if (slot < 0) {  // not resident: a caller error; read slot 0 and report it
+                        atomicOr(err, ERRBIT_STATE);
+                        slot = 0;
+                    }
+                }
+                s_sel_id[lane] = id;
+                s_sel_w[lane] = wv;
+                s_sel_slot[lane] = slot;
+                if (blockIdx.x == 0) {
+                    Ly.ids[lane] = id;
+                    Ly.w[lane] = wv;
+                }
+            }
+        } else if (warp <= 2 && nrows > 0) {
+            // meanwhile warps 1 and 2 take phase C's two units of the shared expert (its h
+            // and its down rows are ready: phase A made them)
+            float hh[D1_HPL];
+            const float4* hv = reinterpret_cast<const float4*>(hsh + lane * D1_HPL);
+#pragma unroll
+            for (int i = 0; i < D1_HPL / 4; ++i) {
+                const float4 v = __ldcg(hv + i);
+                hh[4 * i] = v.x; hh[4 * i + 1] = v.y; hh[4 * i + 2] = v.z; hh[4 * i + 3] = v.w;
+            }
+            unit_dots(k, __ldcg(sgate), hh);
+        }
+        __syncthreads();
+        const int sel_id = lane < k ? s_sel_slot[lane] : 0;  // stack index of selection j
+        const float sel_w = lane < k ? s_sel_w[lane] : 0.0f;
+        if (warp == 0 && nrows > 0) {
+            // phase C's routed down rows do not depend on h: start their copies now
+            for (int j = 0; j < k; ++j) {
+                const int e = __shfl_sync(FULL, sel_id, j);
+                if (lane == 0)
+                    issue_down(j, static_cast<const char*>(Ly.w_down) + size_t(e) * H * drow,
+                               PACKED ? Ly.s_down + size_t(e) * H * (I / 32) : nullptr);
+            }
+        }
+        // the k * I routed gate/up row pairs (u-major)
+        const int J = k * I;
+        auto job_rows = [&](int j, Row& g, Row& u) {
+            const int uu = j / I, i = j - (j / I) * I;
+            const int e = __shfl_sync(FULL, sel_id, uu < k ? uu : 0);
+            if (j < J) {
+                const size_t rowi = size_t(e) * I + i;
+                ld_row<WT>(g, static_cast<const char*>(Ly.w_gate) + rowi * grow,
+                           PACKED ? Ly.s_gate + rowi * (H / 32) : nullptr, H, lane);
+                ld_row<WT>(u, static_cast<const char*>(Ly.w_up) + rowi * grow,
+                           PACKED ? Ly.s_up + rowi * (H / 32) : nullptr, H, lane);
+            }
+        };
+        {
+            // each warp takes the pairs j = gw, gw + Wtot, ... and keeps G of them in flight
+            // (bf16 rows are 4 KB: 2 pairs; packed rows are 1 KB int4 or 512 B int2: all of a
+            // warp's pairs at the Qwen3-Next size, so one memory latency covers them)
+            constexpr int G = WT == DT_BF16 ? D1_G : D1_GQ;
+            const int gw = blockIdx.x * D1_WARPS + warp;
+            for (int jb = gw; jb < J; jb += G * Wtot) {
+                Row g[G], u[G];
+#pragma unroll
+                for (int t = 0; t < G; ++t) job_rows(jb + t * Wtot, g[t], u[t]);
+#pragma unroll
+                for (int t = 0; t < G; ++t) {
+                    const int j = jb + t * Wtot;
+                    if (j < J) {
+                        const float a = hsum2(dot_row<WT>(g[t], xf)), b = hsum2(dot_row<WT>(u[t], xf));
+                        if (lane == 0) p.hrt[j] = silu_mul(a, b);
+                    }
+                }
+            }
+        }
+
+        // ------------------------------------------------------------ phase C
+        grid_barrier(p.ctl, nblocks, bar_idx++, to);
+        if (l + 1 < p.n_layers && threadIdx.x < 32) {
+            // L2 prefetch of the next layer's router rows and shared gate/up rows (the rows
+            // this block streams first in that layer)
+            const DecLayer& Nx = p.L[l + 1];
+            for (int q = lane * nblocks + blockIdx.x; q < E; q += 32 * nblocks)
+                prefetch_l2(static_cast<const char*>(Nx.router_w) + size_t(q) * 2 * H, 2 * H);
+            for (int i = lane * nblocks + blockIdx.x; i < I; i += 32 * nblocks) {
+                prefetch_l2(static_cast<const char*>(Nx.sh_gate) + size_t(i) * grow, grow);
+                prefetch_l2(static_cast<const char*>(Nx.sh_up) + size_t(i) * grow, grow);
+            }
+        }
+        if (nrows > 0) {
+            if (threadIdx.x == 0) {
+                // the routed h rows (written by every block before the barrier) into shared
+                // memory with one bulk copy
+                fence_proxy_async_global();
+                fence_proxy_async_smem();
+                mbar_arrive_expect_tx(hbar, uint32_t(4 * k * I));
+                bulk_g2s(smem + S.hbuf, p.hrt, uint32_t(4 * k * I), hbar);
+            }
+            mbar_wait(hbar, par, err, to);
+#pragma unroll 1
+            for (int m = 0; m < MU; ++m) {
+                const int unit = warp + D1_WARPS * m;
+                if (unit < 2 * k) {
+                    const int u = unit >> 1;
+                    float hh[D1_HPL];
+                    const float4* hv = reinterpret_cast<const float4*>(hbuf + size_t(u) * I + lane * D1_HPL);
+#pragma unroll
+                    for (int i = 0; i < D1_HPL / 4; ++i) {
+                        const float4 v = hv[i];
+                        hh[4 * i] = v.x; hh[4 * i + 1] = v.y; hh[4 * i + 2] = v.z; hh[4 * i + 3] = v.w;
+                    }
+                    unit_dots(u, __shfl_sync(FULL, sel_w, u), hh);
+                }
+            }
         }
         // per row: reduce the lanes, then sum the warps' partials in a fixed order
-        {
-            const int hf = warp & 1;
-            const int ra = hf * half, rn = nrows > 0 ? min(half, nrows - ra) : 0;
 #pragma unroll
-            for (int r = 0; r < D1_RB_MAX / 2; ++r) {
-                const float v = warp_sum(acc[r].x + acc[r].y);
-                if (lane == 0 && r < rn) part[warp * D1_RB_MAX + ra + r] = v;
-            }
+        for (int r = 0; r < D1_RB_MAX / 2; ++r) {
+            const float v = warp_sum(acc[r].x + acc[r].y);
+            if (lane == 0 && r < rn) part[warp * D1_RB_MAX + ra + r] = v;
         }
         __syncthreads();
         if (threadIdx.x < nrows) {
@@ -558,16 +635,16 @@ redmoe_status d1_launch_all(const redmoe_layer* sh, const DecLayer* layers, int 
 
 }  // namespace
 
-// Layers the one-row kernel takes: bf16 x and router, bf16 or int4 experts, the
-// Qwen3-Next expert width (I = Is = 512), H up to 2048 in whole chunks per lane, k up to
-// D1_MAXK, and at most D1_RB_MAX output rows per block.
+// Layers the one-row kernel takes: bf16 x and router, bf16, int4 or int2 experts, the
+// Qwen3-Next expert width (I = Is = 512), H up to 2048 in whole chunks per lane, at most
+// D1_MAXE experts and D1_MAXK per token, and at most D1_RB_MAX output rows per block.
 bool decode1_shape_ok(const redmoe_layer* sh) {
     const int H = sh->hidden, wt = sh->expert_dtype;
     if (sh->x_dtype != DT_BF16 || sh->router_dtype != DT_BF16) return false;
     if (sh->inter != 512 || sh->shared_inter != 512) return false;
     if (wt != DT_BF16 && wt != DT_INT4 && wt != DT_INT2) return false;
     if (H > 32 * D1_XPL || H % (wt == DT_INT2 ? 2048 : (wt == DT_INT4 ? 1024 : 256))) return false;
-    if (sh->top_k > D1_MAXK || sh->n_experts > MAX_EXPERTS) return false;
+    if (sh->top_k > D1_MAXK || sh->n_experts > D1_MAXE) return false;
     return true;
 }
 

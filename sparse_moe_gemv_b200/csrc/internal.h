@@ -46,6 +46,11 @@ struct DecLayer {
     float* out;
     int32_t* ids;
     float* w;
+    // One-row kernel only: routing taken from these arrays instead of computed (NULL:
+    // computed), and routed expert e read from stack index slot_of[e] (NULL: index e).
+    const int32_t* given_ids;
+    const float* given_w;
+    const int32_t* slot_of;
 };
 
 // The decode kernel's view of one redmoe_layer called on (x, out, ids, w).
@@ -76,7 +81,7 @@ redmoe_status launch_decode(const redmoe_layer* shape, const DecLayer* layers, i
 
 // Workspace carve-up of the batched (grouped-GEMM) path (byte offsets from the base).
 struct BatchLayout {
-    size_t logits, sgate, counts, offsets, perm, tiles, bhist, xg, h, total;
+    size_t logits, sgate, counts, offsets, perm, tiles, tiles2, bhist, xg, h, total;
 };
 BatchLayout batch_layout(int T, int E, int k, int H, int I);
 bool batch_shape_ok(const redmoe_layer* L);
