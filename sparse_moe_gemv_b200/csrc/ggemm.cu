@@ -44,20 +44,13 @@ constexpr int RED_COLS = 64;                    // scatter epilogue: columns per
 constexpr int RED_STRIDE = RED_COLS * 4 + 16;   // padded staging row (bytes): 4-way bank conflicts at most
 constexpr int RED_WARP = 2 * 32 * RED_STRIDE;   // two staging buffers of 32 rows per epilogue warp
 
-// MH = 2: a tile of 2 x 128 rows whose two halves share each B tile (two M = 128
-// accumulators side by side in TMEM, all 512 columns at BN = 256, so one accumulator set
-// and no overlap of a tile's epilogue with the next tile's MMAs); MH = 1: 128-row tiles
-// with two accumulator sets in turn.
-template <int MODE, int BN, int MH>
+template <int MODE, int BN>
 struct Cfg {
-    static constexpr int A_HALF = BM * BK * 2;
-    static constexpr int A_BYTES = MH * A_HALF;
+    static constexpr int A_BYTES = BM * BK * 2;
     static constexpr int B_BYTES = BN * BK * 2;
     static constexpr int STAGE = A_BYTES + B_BYTES;
-    static constexpr int NS = (STAGE <= 24 * 1024) ? 8 : (MH == 2 || MODE == GM_SCATTER ? 3 : 4);
-    static constexpr int NACC = MH == 2 ? 1 : 2;  // accumulator sets in TMEM
-    static constexpr int BMT = MH * BM;           // rows of a tile
-    static constexpr int TMEM_COLS = (NACC * MH * BN <= 32) ? 32 : (NACC * MH * BN <= 64 ? 64 : (NACC * MH * BN <= 128 ? 128 : (NACC * MH * BN <= 256 ? 256 : 512)));
+    static constexpr int NS = (STAGE <= 24 * 1024) ? 8 : (MODE == GM_SCATTER ? 3 : 4);
+    static constexpr int TMEM_COLS = (2 * BN <= 32) ? 32 : (2 * BN <= 64 ? 64 : (2 * BN <= 128 ? 128 : (2 * BN <= 256 ? 256 : 512)));
     // scatter: weighted rows for the bulk reductions; router: a 32 x 33 fp32 transpose
     // buffer per epilogue warp
     static constexpr int STAGING = (MODE == GM_SCATTER) ? 4 * RED_WARP : (MODE == GM_ROUTER ? 4 * 32 * 33 * 4 : 0);
@@ -113,9 +106,9 @@ __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" :: "r"(smem_u32(bar)) : "memory");
 }
 
-template <int MODE, int BN, int MH>
+template <int MODE, int BN>
 __global__ void __launch_bounds__(GEMM_THREADS, 1) ggemm_kernel(const __grid_constant__ GemmParams p) {
-    using C = Cfg<MODE, BN, MH>;
+    using C = Cfg<MODE, BN>;
     constexpr int NS = C::NS;
     extern __shared__ unsigned char smem_raw[];
     unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -152,22 +145,16 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) ggemm_kernel(const __grid_con
         uint32_t it = 0;
         for (int w = blockIdx.x; w < total; w += gridDim.x) {
             const Tile t = tile_of<MODE>(p, w);
-            const int rowA = t.S + t.m * C::BMT;
+            const int rowA = t.S + t.m * BM;
             const bool shared = (MODE != GM_ROUTER) && t.g == p.E;
-            const bool two = MH == 2 && t.C - t.m * C::BMT > BM;  // the tile's second half has rows
             for (int kb = 0; kb < p.num_kb; ++kb, ++it) {
                 const int s = int(it % NS);
                 unsigned char* st = smem + s * C::STAGE;
                 if (lane != 0) continue;
                 mbar_wait(empty + s, ((it / NS) & 1u) ^ 1u, err, to);
-                mbar_arrive_expect_tx(full + s, C::STAGE - (MH == 2 && !two ? C::A_HALF : 0));
-                if (MODE == GM_SWIGLU && shared) {
-                    tma_load_2d(st, &p.tmA2, kb * BK, t.m * C::BMT, full + s);
-                    if (two) tma_load_2d(st + C::A_HALF, &p.tmA2, kb * BK, t.m * C::BMT + BM, full + s);
-                } else {
-                    tma_load_2d(st, &p.tmA, kb * BK, rowA, full + s);
-                    if (two) tma_load_2d(st + C::A_HALF, &p.tmA, kb * BK, rowA + BM, full + s);
-                }
+                mbar_arrive_expect_tx(full + s, C::STAGE);
+                if (MODE == GM_SWIGLU && shared) tma_load_2d(st, &p.tmA2, kb * BK, t.m * BM, full + s);
+                else tma_load_2d(st, &p.tmA, kb * BK, rowA, full + s);
                 unsigned char* sb = st + C::A_BYTES;
                 if (MODE == GM_SWIGLU) {
                     const int nh = t.n * (BN / 2);
@@ -192,30 +179,20 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) ggemm_kernel(const __grid_con
         constexpr uint32_t idesc = idesc_bf16_f32(BM, BN);
         uint32_t it = 0, tc = 0;
         for (int w = blockIdx.x; w < total; w += gridDim.x, ++tc) {
-            bool two = false;
-            if (MH == 2) {
-                const Tile t = tile_of<MODE>(p, w);
-                two = t.C - t.m * C::BMT > BM;
-            }
-            const uint32_t acc = tc % C::NACC;
-            mbar_wait(tempty + acc, ((tc / C::NACC) & 1u) ^ 1u, err, to);
+            const uint32_t acc = tc & 1u;
+            mbar_wait(tempty + acc, ((tc >> 1) & 1u) ^ 1u, err, to);
             tc_fence_after();
-            const uint32_t d_tmem = tmem_base + acc * MH * BN;
+            const uint32_t d_tmem = tmem_base + acc * BN;
             for (int kb = 0; kb < p.num_kb; ++kb, ++it) {
                 const int s = int(it % NS);
                 mbar_wait(full + s, (it / NS) & 1u, err, to);
                 tc_fence_after();
                 const uint32_t a_addr = smem_u32(smem + s * C::STAGE);
                 const uint32_t b_addr = a_addr + C::A_BYTES;
-                const uint64_t bd = sw128_kmajor_desc(b_addr);
+                const uint64_t ad = sw128_kmajor_desc(a_addr), bd = sw128_kmajor_desc(b_addr);
 #pragma unroll
-                for (int hh = 0; hh < MH; ++hh) {
-                    if (hh == 1 && !two) break;
-                    const uint64_t ad = sw128_kmajor_desc(a_addr + hh * C::A_HALF);
-#pragma unroll
-                    for (int kk = 0; kk < BK / 16; ++kk)
-                        tc_mma_bf16(d_tmem + hh * BN, ad + uint64_t(2 * kk), bd + uint64_t(2 * kk), idesc, (kb | kk) != 0);
-                }
+                for (int kk = 0; kk < BK / 16; ++kk)
+                    tc_mma_bf16(d_tmem, ad + uint64_t(2 * kk), bd + uint64_t(2 * kk), idesc, (kb | kk) != 0);
                 tc_commit(empty + s);
             }
             tc_commit(tfull + acc);
@@ -235,11 +212,11 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) ggemm_kernel(const __grid_con
         uint32_t red_chunk = 0;              // scatter: staging buffer sequence
         for (int w = blockIdx.x; w < total; w += gridDim.x, ++tc) {
             const Tile t = tile_of<MODE>(p, w);
-            const uint32_t acc = tc % C::NACC;
-            mbar_wait(tfull + acc, (tc / C::NACC) & 1u, err, to);
+            const uint32_t acc = tc & 1u;
+            mbar_wait(tfull + acc, (tc >> 1) & 1u, err, to);
             tc_fence_after();
-            const uint32_t taddr = tmem_base + (uint32_t(q * 32) << 16) + acc * MH * BN;
-            const int lr = t.m * C::BMT + r; // row within the group (first half of the tile)
+            const uint32_t taddr = tmem_base + (uint32_t(q * 32) << 16) + acc * BN;
+            const int lr = t.m * BM + r;     // row within the group
             const bool valid = lr < t.C;
             const int grow = t.S + lr;       // row in the grouped row space
             if (MODE == GM_ROUTER) {
@@ -265,16 +242,12 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) ggemm_kernel(const __grid_con
                     __syncwarp();
                 }
             } else if (MODE == GM_SWIGLU) {
-                const bool two = MH == 2 && t.C - t.m * C::BMT > BM;
 #pragma unroll 1
-                for (int hc = 0; hc < (two ? 2 : 1) * (BN / 64); ++hc) {
-                    const int hh = hc / (BN / 64), c = hc - hh * (BN / 64);  // tile half, column chunk
-                    const int lrh = lr + hh * BM;
-                    const int growh = grow + hh * BM;
+                for (int c = 0; c < BN / 64; ++c) {
                     float g[32], u[32];
-                    tmem_ld32(taddr + hh * BN + c * 32, g);
-                    tmem_ld32(taddr + hh * BN + BN / 2 + c * 32, u);
-                    if (lrh < t.C) {
+                    tmem_ld32(taddr + c * 32, g);
+                    tmem_ld32(taddr + BN / 2 + c * 32, u);
+                    if (valid) {
                         uint32_t pk[16];
 #pragma unroll
                         for (int j = 0; j < 16; ++j) {
@@ -282,7 +255,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) ggemm_kernel(const __grid_con
                             const float h1 = g[2 * j + 1] / (1.0f + expf(-g[2 * j + 1])) * u[2 * j + 1];
                             pk[j] = uint32_t(f2bf(h0)) | (uint32_t(f2bf(h1)) << 16);
                         }
-                        uint4* dst = reinterpret_cast<uint4*>(p.out_bf16 + size_t(growh) * p.N + t.n * (BN / 2) + c * 32);
+                        uint4* dst = reinterpret_cast<uint4*>(p.out_bf16 + size_t(grow) * p.N + t.n * (BN / 2) + c * 32);
 #pragma unroll
                         for (int j = 0; j < 4; ++j) dst[j] = make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
                     }
@@ -351,7 +324,7 @@ EncodeTiledFn encode_fn() {
     return fn;
 }
 
-template <int MODE, int BN, int MH>
+template <int MODE, int BN>
 int blocks_for(const void* kern, int smem) {
     static std::mutex mu;
     static std::vector<int> done;
@@ -366,14 +339,14 @@ int blocks_for(const void* kern, int smem) {
     return 1;
 }
 
-template <int MODE, int BN, int MH>
+template <int MODE, int BN>
 redmoe_status launch_gemm(GemmParams& p, cudaStream_t stream) {
-    using C = Cfg<MODE, BN, MH>;
+    using C = Cfg<MODE, BN>;
     DevInfo di;
     if (!get_dev_info(&di)) return REDMOE_ERR_CUDA;
     if (C::SMEM > di.max_smem_optin) return REDMOE_ERR_UNSUPPORTED;
-    auto kern = ggemm_kernel<MODE, BN, MH>;
-    if (blocks_for<MODE, BN, MH>(reinterpret_cast<const void*>(kern), C::SMEM) < 0) return REDMOE_ERR_CUDA;
+    auto kern = ggemm_kernel<MODE, BN>;
+    if (blocks_for<MODE, BN>(reinterpret_cast<const void*>(kern), C::SMEM) < 0) return REDMOE_ERR_CUDA;
     p.timeout_ns = BARRIER_TIMEOUT_NS;
     kern<<<di.sm_count, GEMM_THREADS, C::SMEM, stream>>>(p);
     return cudaGetLastError() == cudaSuccess ? REDMOE_OK : REDMOE_ERR_CUDA;
@@ -395,9 +368,8 @@ bool make_tmap_bf16(CUtensorMap* m, const void* base, uint64_t rows, uint64_t K,
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-redmoe_status gemm_router(GemmParams& p, cudaStream_t s) { return launch_gemm<GM_ROUTER, 64, 1>(p, s); }
-// gate/up: 256-row tiles (p.tiles counts 256-row m-tiles per group)
-redmoe_status gemm_swiglu(GemmParams& p, cudaStream_t s) { return launch_gemm<GM_SWIGLU, 256, 2>(p, s); }
-redmoe_status gemm_scatter(GemmParams& p, cudaStream_t s) { return launch_gemm<GM_SCATTER, 256, 1>(p, s); }
+redmoe_status gemm_router(GemmParams& p, cudaStream_t s) { return launch_gemm<GM_ROUTER, 64>(p, s); }
+redmoe_status gemm_swiglu(GemmParams& p, cudaStream_t s) { return launch_gemm<GM_SWIGLU, 256>(p, s); }
+redmoe_status gemm_scatter(GemmParams& p, cudaStream_t s) { return launch_gemm<GM_SCATTER, 256>(p, s); }
 
 }  // namespace redmoe

@@ -81,7 +81,7 @@ redmoe_status launch_decode(const redmoe_layer* shape, const DecLayer* layers, i
 
 // Workspace carve-up of the batched (grouped-GEMM) path (byte offsets from the base).
 struct BatchLayout {
-    size_t logits, sgate, counts, offsets, perm, tiles, tiles2, bhist, xg, h, total;
+    size_t logits, sgate, counts, offsets, perm, tiles, bhist, xg, h, total;
 };
 BatchLayout batch_layout(int T, int E, int k, int H, int I);
 bool batch_shape_ok(const redmoe_layer* L);

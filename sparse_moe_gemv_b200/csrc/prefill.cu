@@ -32,8 +32,8 @@ redmoe_status gemm_swiglu(GemmParams& p, cudaStream_t s);
 redmoe_status gemm_scatter(GemmParams& p, cudaStream_t s);
 redmoe_status launch_route(const redmoe_layer* L, const void* x, int T, const float* logits, int32_t* ids, float* w,
                            float* sgate, int32_t* counts, int32_t* offsets, int32_t* perm, int tile_m,
-                           int32_t* tiles, int tile_m2, int32_t* tiles2, void* xg, int32_t* bhist, Control* ctl,
-                           cudaStream_t stream, int* launches, CacheBias cb);
+                           int32_t* tiles, void* xg, int32_t* bhist, Control* ctl, cudaStream_t stream,
+                           int* launches, CacheBias cb);
 
 BatchLayout batch_layout(int T, int E, int k, int H, int I) {
     BatchLayout b;
@@ -45,7 +45,6 @@ BatchLayout batch_layout(int T, int E, int k, int H, int I) {
     b.offsets = o; o = align256(o + 4ull * (E + 1));
     b.perm = o; o = align256(o + 4ull * T * k);
     b.tiles = o; o = align256(o + 4ull * (E + 2));
-    b.tiles2 = o; o = align256(o + 4ull * (E + 2));
     b.bhist = o; o = align256(o + 4ull * ROUTE_MAX_BLOCKS * E);
     b.xg = o; o = align256(o + 2ull * T * k * H);
     b.h = o; o = align256(o + 2ull * rows * I);
@@ -70,7 +69,6 @@ redmoe_status launch_batched(const redmoe_layer* L, const void* x, int T, float*
     int32_t* offsets = reinterpret_cast<int32_t*>(base + B.offsets);
     int32_t* perm = reinterpret_cast<int32_t*>(base + B.perm);
     int32_t* tiles = reinterpret_cast<int32_t*>(base + B.tiles);
-    int32_t* tiles2 = reinterpret_cast<int32_t*>(base + B.tiles2);
     int32_t* bhist = reinterpret_cast<int32_t*>(base + B.bhist);
     Control* ctl = reinterpret_cast<Control*>(base);
     void* xg = base + B.xg;
@@ -88,8 +86,8 @@ redmoe_status launch_batched(const redmoe_layer* L, const void* x, int T, float*
     if ((st = gemm_router(gr, s)) != REDMOE_OK) return st;
     if (launches) *launches += 1;
     // 2 routing: top-k, weights, shared gate, zeroed out, grouping, tile schedule, gathered x
-    if ((st = launch_route(L, x, T, logits, ids, w, sgate, counts, offsets, perm, 128, tiles, 256, tiles2, xg, bhist,
-                           ctl, s, launches, cb)) != REDMOE_OK)
+    if ((st = launch_route(L, x, T, logits, ids, w, sgate, counts, offsets, perm, 128, tiles, xg, bhist, ctl, s,
+                           launches, cb)) != REDMOE_OK)
         return st;
     if (dbg) {
         if (cudaMemcpyAsync(dbg->counts, counts, 4ull * E, cudaMemcpyDeviceToDevice, s) != cudaSuccess ||
@@ -105,7 +103,7 @@ redmoe_status launch_batched(const redmoe_layer* L, const void* x, int T, float*
         !make_tmap_bf16(&g1.tmS0, L->sh_gate, I, H, 128) || !make_tmap_bf16(&g1.tmS1, L->sh_up, I, H, 128))
         return REDMOE_ERR_CUDA;
     g1.E = E; g1.T = T; g1.k = k; g1.N = I; g1.Nb = I; g1.n_tiles = I / 128; g1.num_kb = H / 64;
-    g1.offsets = offsets; g1.tiles = tiles2; g1.out_bf16 = hbuf; g1.ctl = ctl;  // 256-row tiles
+    g1.offsets = offsets; g1.tiles = tiles; g1.out_bf16 = hbuf; g1.ctl = ctl;
     if ((st = gemm_swiglu(g1, s)) != REDMOE_OK) return st;
     if (launches) *launches += 1;
     // 4 down + weighted scatter-add into out

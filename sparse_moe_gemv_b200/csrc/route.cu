@@ -41,9 +41,7 @@ struct RouteParams {
     int32_t* offsets;     // [E + 1]
     int32_t* perm;        // [T * k]
     int tile_m;
-    int32_t* tiles;       // [E + 2] prefix of tile_m-row tiles per group (the shared expert last)
-    int tile_m2;
-    int32_t* tiles2;      // [E + 2] the same for tile_m2-row tiles
+    int32_t* tiles;       // [E + 2]
     uint16_t* xg;         // [T * k, H] bf16 gathered rows
     int32_t* bhist;       // [grid, E]
     Control* ctl;
@@ -189,20 +187,16 @@ __global__ void __launch_bounds__(RT_THREADS, 1) route_kernel(const __grid_const
     for (int e = threadIdx.x; e < E; e += RT_THREADS) hist[e] = offs[e] + __ldcg(p.bhist + size_t(blockIdx.x) * E + e);
     if (blockIdx.x == 0) {
         for (int e = threadIdx.x; e <= E; e += RT_THREADS) p.offsets[e] = offs[e];
-        for (int pass = 0; pass < 2; ++pass) {
-            const int tm = pass == 0 ? p.tile_m : p.tile_m2;
-            int32_t* out = pass == 0 ? p.tiles : p.tiles2;
-            if (tm <= 0) continue;
-            for (int e = threadIdx.x; e < E; e += RT_THREADS) tmp[e] = (__ldcg(p.counts + e) + tm - 1) / tm;
+        if (p.tile_m > 0) {
+            for (int e = threadIdx.x; e < E; e += RT_THREADS) tmp[e] = (__ldcg(p.counts + e) + p.tile_m - 1) / p.tile_m;
             __syncthreads();
             int* tl = tmp;  // scanned in place
             const int nt = block_scan2(tmp, tl, E, wsum);
-            for (int e = threadIdx.x; e < E; e += RT_THREADS) out[e] = tl[e];
+            for (int e = threadIdx.x; e < E; e += RT_THREADS) p.tiles[e] = tl[e];
             if (threadIdx.x == 0) {
-                out[E] = nt;
-                out[E + 1] = nt + (T + tm - 1) / tm;
+                p.tiles[E] = nt;
+                p.tiles[E + 1] = nt + (T + p.tile_m - 1) / p.tile_m;
             }
-            __syncthreads();
         }
     }
     __syncthreads();
@@ -265,8 +259,8 @@ int route_smem_bytes(int E, int tpb, int k) { return 4 * (3 * E + 1 + 32 + 2 * t
 
 redmoe_status launch_route(const redmoe_layer* L, const void* x, int T, const float* logits, int32_t* ids, float* w,
                            float* sgate, int32_t* counts, int32_t* offsets, int32_t* perm, int tile_m,
-                           int32_t* tiles, int tile_m2, int32_t* tiles2, void* xg, int32_t* bhist, Control* ctl,
-                           cudaStream_t stream, int* launches, CacheBias cb) {
+                           int32_t* tiles, void* xg, int32_t* bhist, Control* ctl, cudaStream_t stream,
+                           int* launches, CacheBias cb) {
     DevInfo di;
     if (!get_dev_info(&di)) return REDMOE_ERR_CUDA;
     const int E = L->n_experts, k = L->top_k;
@@ -279,7 +273,6 @@ redmoe_status launch_route(const redmoe_layer* L, const void* x, int T, const fl
     p.tpb = (T + nb - 1) / nb;
     p.ids = ids; p.w = w; p.sgate = sgate;
     p.counts = counts; p.offsets = offsets; p.perm = perm; p.tile_m = tile_m; p.tiles = tiles;
-    p.tile_m2 = tile_m2; p.tiles2 = tiles2;
     p.xg = static_cast<uint16_t*>(xg); p.bhist = bhist; p.ctl = ctl; p.timeout_ns = BARRIER_TIMEOUT_NS;
     p.cb = cb;
     const int smem = route_smem_bytes(E, p.tpb, k);
