@@ -758,8 +758,8 @@ def run_sub_workload(args, name):
     """One extra workload of the default line, in a child process with a CUDA context of its
     own, so that the workloads share no device state; returns (object, cpu-baseline extras)."""
     import subprocess
-    cmd = [sys.executable, os.path.abspath(__file__), "--workload", name, "--steps", str(min(args.steps, SUB_STEPS[name])),
-           "--warmup", "3", "--sub"]
+    steps = SUB_STEPS[name] if name == "hostexp" else min(args.steps, SUB_STEPS[name])  # hostexp: its whole stream
+    cmd = [sys.executable, os.path.abspath(__file__), "--workload", name, "--steps", str(steps), "--warmup", "3", "--sub"]
     if not args.no_cpu_baseline:
         cmd.append("--sub-cpu")
     r = subprocess.run(cmd, capture_output=True, text=True, timeout=900)
