@@ -811,6 +811,7 @@ bool decode_shape_ok(const redmoe_layer* sh) {
 redmoe_status launch_decode(const redmoe_layer* sh, const DecLayer* layers, int n_layers, int T, void* ws,
                             cudaStream_t stream, int* launches, CacheBias cb) {
     if (T == 1 && decode1_shape_ok(sh)) return launch_decode1(sh, layers, n_layers, ws, stream, launches, cb);
+    if (decodefr_shape_ok(sh, T)) return launch_decodefr(sh, layers, n_layers, T, ws, stream, launches, cb);
     if (!decode_shape_ok(sh)) return REDMOE_ERR_UNSUPPORTED;
     const int xt = sh->x_dtype, rt = sh->router_dtype, wt = sh->expert_dtype;
     if (xt == DT_F32 && rt == DT_F32 && wt == DT_F32)

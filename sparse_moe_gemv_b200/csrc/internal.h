@@ -75,6 +75,11 @@ bool decode1_shape_ok(const redmoe_layer* sh);
 redmoe_status launch_decode1(const redmoe_layer* sh, const DecLayer* layers, int n_layers, void* ws,
                              cudaStream_t stream, int* launches, CacheBias cb);
 
+// The few-row kernel (T = 2, 3; bf16 or int4 experts of the Qwen3-Next width).
+bool decodefr_shape_ok(const redmoe_layer* sh, int T);
+redmoe_status launch_decodefr(const redmoe_layer* sh, const DecLayer* layers, int n_layers, int T, void* ws,
+                              cudaStream_t stream, int* launches, CacheBias cb);
+
 // Launch the persistent decode kernel over n_layers layers (1..MAX_STACK).
 redmoe_status launch_decode(const redmoe_layer* shape, const DecLayer* layers, int n_layers, int T,
                             void* workspace, cudaStream_t stream, int* launches, CacheBias cb = CacheBias{nullptr, 0.0f});
