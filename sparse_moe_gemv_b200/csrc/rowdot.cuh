@@ -199,5 +199,93 @@ __host__ __device__ constexpr int d1_row_bytes(int wt, int K) {
 __host__ __device__ constexpr int d1_scale_bytes(int wt, int K) { return wt == DT_BF16 ? 0 : K / 16; }
 
 
+// x rows as packed bf16 pairs in the layout of weight type W: word m of row t is
+// elements 2m, 2m + 1 of the lane's slice (bf16: chunk c = lane + 32 j covers elements
+// 8c .. 8c + 7 -> words 4j .. 4j + 3; int4: chunk c covers 32c .. 32c + 31 -> words
+// 16j .. 16j + 15).
+template <int W, int T>
+__device__ __forceinline__ void load_xp(const uint16_t* x, int H, int lane, uint32_t (&xp)[T][32]) {
+    constexpr int PER = ChunkElems<W>::n;
+    constexpr int NJ = D1_XPL / PER;
+#pragma unroll
+    for (int t = 0; t < T; ++t) {
+#pragma unroll
+        for (int j = 0; j < NJ; ++j) {
+            const int c = lane + 32 * j;
+#pragma unroll
+            for (int q = 0; q < PER / 8; ++q) {
+                const int idx = c * PER + q * 8;
+                const uint4 v = idx < H ? __ldg(reinterpret_cast<const uint4*>(x + size_t(t) * H + idx))
+                                        : make_uint4(0u, 0u, 0u, 0u);
+                const int w = (j * (PER / 8) + q) * 4;
+                xp[t][w] = v.x;
+                xp[t][w + 1] = v.y;
+                xp[t][w + 2] = v.z;
+                xp[t][w + 3] = v.w;
+            }
+        }
+    }
+}
+
+// A packed bf16 pair of x widened to fp32 where it is used: the conversion is kept inside
+// the loop (volatile), so the compiler does not hoist the widened copies of all T rows of
+// x out of phase B's loop and run out of registers.
+__device__ __forceinline__ float2 bf2x(uint32_t w) {
+    uint32_t lo, hi;
+    asm volatile("shl.b32 %0, %2, 16;\n\tand.b32 %1, %2, 0xffff0000;" : "=r"(lo), "=r"(hi) : "r"(w));
+    return make_float2(__uint_as_float(lo), __uint_as_float(hi));
+}
+
+// acc[t] += row . x_t for the rows t with bit t of `mask`
+template <int T>
+__device__ __forceinline__ void dotT_bf(const RowBF& r, const uint32_t (&xp)[T][32], unsigned mask, float2 (&acc)[T]) {
+#pragma unroll
+    for (int j = 0; j < D1_XPL / 8; ++j) {
+        const float2 w0 = bf2(r.w[j].x), w1 = bf2(r.w[j].y), w2 = bf2(r.w[j].z), w3 = bf2(r.w[j].w);
+#pragma unroll
+        for (int t = 0; t < T; ++t) {
+            if (mask >> t & 1u) {
+                float2 a = acc[t];
+                a = ffma2(w0, bf2x(xp[t][4 * j]), a);
+                a = ffma2(w1, bf2x(xp[t][4 * j + 1]), a);
+                a = ffma2(w2, bf2x(xp[t][4 * j + 2]), a);
+                acc[t] = ffma2(w3, bf2x(xp[t][4 * j + 3]), a);
+            }
+        }
+    }
+}
+template <int T>
+__device__ __forceinline__ void dotT_q4(const RowQ4& r, const uint32_t (&xp)[T][32], unsigned mask, float2 (&acc)[T]) {
+    const float2 off = make_float2(-8388616.0f, -8388616.0f);  // -(2^23 + 8)
+#pragma unroll
+    for (int j = 0; j < D1_XPL / 32; ++j) {
+        const uint32_t w[4] = {r.w[j].x, r.w[j].y, r.w[j].z, r.w[j].w};
+        float2 d[T];
+#pragma unroll
+        for (int t = 0; t < T; ++t) d[t] = make_float2(0.f, 0.f);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const uint32_t lo = w[q] & 0x0F0F0F0Fu, hi = (w[q] >> 4) & 0x0F0F0F0Fu;
+#pragma unroll
+            for (uint32_t b = 0; b < 4; ++b) {
+                const float2 wf = fadd2(make_float2(code_f(lo, b), code_f(hi, b)), off);
+#pragma unroll
+                for (int t = 0; t < T; ++t)
+                    if (mask >> t & 1u) d[t] = ffma2(wf, bf2x(xp[t][16 * j + 4 * q + b]), d[t]);
+            }
+        }
+        const float s = bf16f(r.s[j]);
+#pragma unroll
+        for (int t = 0; t < T; ++t)
+            if (mask >> t & 1u) acc[t] = ffma2(make_float2(s, s), d[t], acc[t]);
+    }
+}
+template <int W, int T>
+__device__ __forceinline__ void dotT(const typename RowOf<W>::type& r, const uint32_t (&xp)[T][32], unsigned mask,
+                                     float2 (&acc)[T]) {
+    if constexpr (W == DT_INT4) dotT_q4<T>(r, xp, mask, acc);
+    else dotT_bf<T>(r, xp, mask, acc);
+}
+
 }  // namespace
 }  // namespace redmoe
