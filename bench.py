@@ -53,13 +53,13 @@ QWEN_INT2 = mi.LayerShape(H=2048, E=512, k=10, I=512, Is=512, expert_dtype="int2
 QWEN_ZIPF = mi.LayerShape(H=2048, E=512, k=10, I=512, Is=512, zipf_s=1.1)
 
 WORKLOADS = {
-    "decode_t1": dict(shape=QWEN, T=1, layers=12, stack=False, seed=1000, kernel="decode_kernel",
+    "decode_t1": dict(shape=QWEN, T=1, layers=12, stack=False, seed=1000, kernel="decode1_kernel",
                       desc="Qwen3-Next-shaped MoE layer, bf16 weights / fp32 accumulate, decode T=1"),
-    "fewrow_t2": dict(shape=QWEN, T=2, layers=12, stack=True, seed=2000, kernel="decode_kernel",
+    "fewrow_t2": dict(shape=QWEN, T=2, layers=12, stack=True, seed=2000, kernel="decodefr_kernel",
                       desc="12 distinct Qwen3-Next-shaped bf16 layers back to back, T=2"),
     "fewrow_t3": dict(shape=QWEN, T=3, layers=12, stack=True, seed=2000, kernel="decode_kernel",
                       desc="12 distinct Qwen3-Next-shaped bf16 layers back to back, T=3"),
-    "int4_48": dict(shape=QWEN_INT4, T=1, layers=48, stack=True, seed=4000, kernel="decode_kernel",
+    "int4_48": dict(shape=QWEN_INT4, T=1, layers=48, stack=True, seed=4000, kernel="decode1_kernel",
                     desc="48 distinct Qwen3-Next-shaped layers, int4 group-32 experts, decode T=1"),
     "int2_48": dict(shape=QWEN_INT2, T=1, layers=48, stack=True, seed=5000, kernel="decode1_kernel",
                     desc="48 distinct Qwen3-Next-shaped layers, int2 group-32 experts, decode T=1"),
@@ -122,7 +122,8 @@ def layer_call_bytes(shape, T, distinct):
 
 # kernel sources behind each path: a committed DRAM-traffic figure stays valid while these
 # files are unchanged
-DECODE_SOURCES = ["common.cuh", "decode.cu", "gemv.cuh", "internal.h", "topk.cuh"]
+DECODE_SOURCES = ["common.cuh", "decode.cu", "decode1.cu", "decode_fr.cu", "gemv.cuh", "internal.h", "rowdot.cuh",
+                  "topk.cuh"]
 PREFILL_SOURCES = ["common.cuh", "ggemm.cu", "ggemm_params.h", "internal.h", "prefill.cu", "route.cu", "tc.cuh", "topk.cuh"]
 
 
@@ -134,9 +135,10 @@ def source_digest(files):
     return h.hexdigest()[:16]
 
 
-def profile_traffic(workload):
+def profile_traffic(workload, layers_per_launch=1):
     """DRAM bytes per launch (per step for the batched layer) from the committed ncu summary,
-    if it was taken on the current kernel sources."""
+    if it was taken on the current kernel sources. A layer stack's figure is stored per layer
+    (captured on a shorter stack of the same layers) and scaled by the layers of one launch."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
         return None
@@ -144,6 +146,8 @@ def profile_traffic(workload):
     files = PREFILL_SOURCES if workload.startswith("prefill") else DECODE_SOURCES
     if not d or d.get("source_digest") != source_digest(files):
         return None
+    if "dram_bytes_per_layer" in d:
+        return d["dram_bytes_per_layer"] * layers_per_launch
     return d.get("dram_bytes_per_launch")
 
 
@@ -511,7 +515,8 @@ def gpu_arm(args, wl, world, rank, local, B=None, name=None):
         launches = K * 4
     else:
         roof = {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
-                "traffic": profile_traffic(key), "kernel": wl["kernel"], "bytes_per_launch": bytes_per_launch,
+                "traffic": profile_traffic(key, wl["layers"] if wl["stack"] else 1), "kernel": wl["kernel"],
+                "bytes_per_launch": bytes_per_launch,
                 "launch_us": launch_s * 1e6, "distinct_experts_per_layer": statistics.mean(distinct),
                 "peak_source": f"{src} (MEASURED_PEAKS.json hbm_gbs)" if src == "measured" else "fallback"}
 
