@@ -76,7 +76,13 @@ def test_traffic_figure_needs_matching_sources(bench, tmp_path, monkeypatch):
     for wl, d in committed.items():
         files = bench.PREFILL_SOURCES if wl.startswith("prefill") else bench.DECODE_SOURCES
         current = d["source_digest"] == bench.source_digest(files)
-        assert bench.profile_traffic(wl) == (d["dram_bytes_per_launch"] if current else None), wl
+        if "dram_bytes_per_layer" in d:
+            # a stack's figure is per layer, scaled by the layers of one launch
+            want = d["dram_bytes_per_layer"] * bench.WORKLOADS[wl]["layers"]
+            got = bench.profile_traffic(wl, bench.WORKLOADS[wl]["layers"])
+        else:
+            want, got = d["dram_bytes_per_launch"], bench.profile_traffic(wl)
+        assert got == (want if current else None), wl
     # a workload without a capture reports none
     assert bench.profile_traffic("prefill_uniform") is None
     # a figure taken on other sources is not reported
