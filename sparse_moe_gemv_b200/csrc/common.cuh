@@ -220,6 +220,29 @@ __device__ __forceinline__ void grid_wait(Control* ctl, unsigned nblocks, unsign
     __syncthreads();
 }
 
+// grid_wait for the calling warp alone: lane 0 waits (same bound and error report), then
+// the warp's lanes see what every block wrote before its arrive. The block's other warps
+// are not held.
+__device__ __forceinline__ void grid_wait_warp(Control* ctl, unsigned nblocks, unsigned index, uint64_t timeout_ns) {
+    if ((threadIdx.x & 31) == 0) {
+        const unsigned target = (index + 1u) * nblocks;
+        if (ld_acquire_gpu(&ctl->bar_count) < target) {
+            const uint64_t t0 = globaltimer_ns();
+            for (uint32_t spins = 1; ld_acquire_gpu(&ctl->bar_count) < target; ++spins) {
+                if ((spins & 63u) == 0u) {
+                    const uint64_t dt = globaltimer_ns() - t0;
+                    if (dt > timeout_ns || spins > (1u << 26) || (dt > 20000u && ld_relaxed_gpu(&ctl->err) != 0)) {
+                        atomicOr(&ctl->err, ERRBIT_TIMEOUT);
+                        break;
+                    }
+                }
+            }
+        }
+        __threadfence();
+    }
+    __syncwarp();
+}
+
 // End of a launch that used grid_barrier: the last block out resets the counters.
 __device__ __forceinline__ void grid_exit(Control* ctl, unsigned nblocks) {
     __syncthreads();

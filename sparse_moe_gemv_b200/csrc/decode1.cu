@@ -6,25 +6,28 @@
 // dependent steps (router -> routed gate/up -> down) and how fast each one reaches full
 // bandwidth. This kernel is organised around that:
 //
-//   * Every lane keeps its slice of x in registers as fp32 for the whole layer, so a weight
-//     chunk is dotted straight out of the registers it was loaded into: no shared-memory
-//     traffic for activations or for gate/up weights.
+//   * x is bulk-copied into shared memory once per layer; every lane keeps its slice in
+//     registers as fp32 while it streams rows, so a weight chunk is dotted straight out of
+//     the registers it was loaded into: no shared-memory traffic for gate/up weights.
 //   * Phase A: warps stream the router rows and the shared-gate row with 16-byte vector
-//     loads. Meanwhile one thread per block starts a bulk copy of the block's rows of the
-//     shared expert's down matrix into shared memory.
-//   * Grid barrier; one warp per block computes the top-k of the 512 logits in registers
-//     (router, top-k and shared gate form one stage: "Research notes, October 2026",
-//     section 1) while the other warps stream the shared expert's gate/up rows (the
-//     shared expert needs no routing: the "extra slot" of the DwarfStar MoE kernel, same
-//     section). Then one thread per block starts bulk copies of the block's rows of the k
-//     routed experts' down matrices: phase C's weights stream into shared memory during
-//     phase B, since they do not depend on h.
+//     loads, and nothing else: they are all that stands between the launch and the top-k.
+//     Meanwhile one thread per block starts a bulk copy of the block's rows of the shared
+//     expert's down matrix into shared memory.
+//   * Split grid barrier: each block publishes its logits (arrive); then warps 1..7
+//     stream the block's share of the shared expert's gate/up rows (the shared expert
+//     needs no routing: the "extra slot" of the DwarfStar MoE kernel, "Research notes,
+//     October 2026", section 1) while warp 0 alone waits for the other blocks.
+//   * Warp 0 computes the top-k of the 512 logits in registers (router, top-k and shared
+//     gate form one stage: same section). Then one thread per block starts bulk
+//     copies of the block's rows of the k routed experts' down matrices: phase C's weights
+//     stream into shared memory during phase B, since they do not depend on h.
 //   * Phase B: the k * I routed gate/up row pairs, interleaved over all warps; bf16 warps
 //     keep two pairs of loads in flight, int4/int2 warps issue all of theirs at once;
 //     h = silu(a) * u.
-//   * Grid barrier; h is bulk-copied into shared memory and phase C computes the block's
-//     output rows from the down rows already there. Each output row is summed over the
-//     experts in a fixed order: the result is deterministic.
+//   * Grid barrier; the routed and shared h rows are bulk-copied into shared memory and
+//     phase C computes the block's output rows from the down rows already there (the
+//     shared expert is slot k). Each output row is summed over the experts in a fixed
+//     order: the result is deterministic.
 //
 // Down rows are only I = 512 elements long (1 KiB bf16, 256 B + 32 B int4): the block's
 // rows of one expert form one contiguous range, copied in one piece, which is the lesson
@@ -49,17 +52,18 @@ __device__ __forceinline__ float hsum2(float2 v) { return warp_sum(v.x + v.y); }
 // down matrix of k + 1 experts (routed slots 0..k-1 in selection order, the shared
 // expert in slot k), each slot RB rows (int4: codes, then scales).
 struct D1Smem {
-    int dreg, slot, sc_off, hbuf, bars, part, sel, total;
+    int dreg, slot, sc_off, hbuf, xs, bars, part, sel, total;
 };
-__host__ __device__ inline D1Smem d1_smem(int wt, int k, int I, int RB) {
+__host__ __device__ inline D1Smem d1_smem(int wt, int k, int I, int RB, int H) {
     D1Smem s;
     const int drow = d1_row_bytes(wt, I);
     s.sc_off = a16(RB * drow);
     s.slot = a16(s.sc_off + RB * d1_scale_bytes(wt, I));
     int o = 0;
     s.dreg = o; o += (k + 1) * s.slot;
-    s.hbuf = o; o += a16(4 * k * I);  // the routed h rows, staged for phase C
-    s.bars = o; o += 8 * (D1_MAXK + 2);
+    s.hbuf = o; o += a16(4 * (k + 1) * I);  // the routed and the shared h rows, staged for phase C
+    s.xs = o; o += a16(2 * H);  // the layer's x (bf16), one bulk copy per layer
+    s.bars = o; o += 8 * (D1_MAXK + 3);
     s.part = o; o += 4 * D1_WARPS * D1_RB_MAX;
     s.sel = o; o += 12 * D1_MAXK;  // the block's top-k: ids, weights, stack indices
     s.total = a16(o);
@@ -89,10 +93,11 @@ __global__ void __launch_bounds__(D1_THREADS, 1) decode1_kernel(const __grid_con
     const int Wtot = nblocks * D1_WARPS;
     int* err = &p.ctl->err;
     const uint64_t to = p.timeout_ns;
-    const D1Smem S = d1_smem(WT, k, I, RB);
+    const D1Smem S = d1_smem(WT, k, I, RB, H);
     unsigned char* dreg = smem + S.dreg;
     uint64_t* dbar = reinterpret_cast<uint64_t*>(smem + S.bars);
     uint64_t* hbar = dbar + D1_MAXK + 1;
+    uint64_t* xbar = dbar + D1_MAXK + 2;
     const float* hbuf = reinterpret_cast<const float*>(smem + S.hbuf);
     float* part = reinterpret_cast<float*>(smem + S.part);
     int* s_sel_id = reinterpret_cast<int*>(smem + S.sel);
@@ -109,6 +114,7 @@ __global__ void __launch_bounds__(D1_THREADS, 1) decode1_kernel(const __grid_con
     if (threadIdx.x == 0) {
         for (int i = 0; i <= k; ++i) mbar_init(dbar + i, 1);
         mbar_init(hbar, 1);
+        mbar_init(xbar, 1);
         fence_mbar_init();
     }
     __syncthreads();
@@ -130,52 +136,59 @@ __global__ void __launch_bounds__(D1_THREADS, 1) decode1_kernel(const __grid_con
         const uint32_t par = uint32_t(l & 1);
 
         // ------------------------------------------------------------ phase A
-        if (threadIdx.x == 0 && nrows > 0) {
-            fence_proxy_async_smem();  // the previous layer's reads of dreg come first
-            issue_down(k, Ly.sh_down, Ly.sh_s_down);
+        if (threadIdx.x == 0) {
+            fence_proxy_async_smem();  // the previous layer's reads of dreg and xs come first
+            mbar_arrive_expect_tx(xbar, uint32_t(2 * H));
+            bulk_g2s(smem + S.xs, x, uint32_t(2 * H), xbar);
+            if (nrows > 0) issue_down(k, Ly.sh_down, Ly.sh_s_down);
         }
-        // job q < E: router row q; q == E: shared-gate row; q > E: the shared expert's
-        // gate/up row q - E - 1 (it needs no routing: the extra expert slot of the DwarfStar
-        // MoE kernel). Warp w of block b takes q = w * nblocks + b (+ Wtot ...): the router
-        // rows go to the low warps of every block, the shared rows to the others.
-        for (int q = warp * nblocks + blockIdx.x; q < E + 1 + I; q += Wtot) {
+        // job q < E: router row q; q == E: shared-gate row. Warp w of block b takes
+        // q = w * nblocks + b: the jobs go to the low warps of every block. Only these rows
+        // stand between the launch and the top-k, so nothing else is streamed before them.
+        for (int q = warp * nblocks + blockIdx.x; q < E + 1; q += Wtot) {
             if (Ly.given_ids && q < E) continue;  // routing given: no router rows
             float xr[D1_XPL];
-            if (q <= E) {
-                RowBF r;
-                const void* row = q < E ? static_cast<const void*>(static_cast<const char*>(Ly.router_w) + size_t(q) * 2 * H)
-                                        : Ly.shared_gate_w;
-                ld_row_bf(r, row, H, lane);
-                load_x<DT_BF16>(x, H, lane, xr);
-                const float v = hsum2(dot_row_bf(r, xr));
-                if (lane == 0) {
-                    if (q < E) p.logits[q] = v + (Ly.router_bias ? Ly.router_bias[q] : 0.0f);
-                    else *sgate = 1.0f / (1.0f + expf(-v));
-                }
-            } else {
-                const int i = q - E - 1;
-                Row g, u;
-                ld_row<WT>(g, static_cast<const char*>(Ly.sh_gate) + size_t(i) * grow,
-                           PACKED ? Ly.sh_s_gate + size_t(i) * (H / 32) : nullptr, H, lane);
-                ld_row<WT>(u, static_cast<const char*>(Ly.sh_up) + size_t(i) * grow,
-                           PACKED ? Ly.sh_s_up + size_t(i) * (H / 32) : nullptr, H, lane);
-                load_x<WT>(x, H, lane, xr);
-                const float a = hsum2(dot_row<WT>(g, xr)), b = hsum2(dot_row<WT>(u, xr));
-                if (lane == 0) hsh[i] = silu_mul(a, b);
+            RowBF r;
+            const void* row = q < E ? static_cast<const void*>(static_cast<const char*>(Ly.router_w) + size_t(q) * 2 * H)
+                                    : Ly.shared_gate_w;
+            ld_row_bf(r, row, H, lane);
+            mbar_wait(xbar, par, err, to);
+            load_x<DT_BF16, true>(reinterpret_cast<const uint16_t*>(smem + S.xs), H, lane, xr);
+            const float v = hsum2(dot_row_bf(r, xr));
+            if (lane == 0) {
+                if (q < E) p.logits[q] = v + (Ly.router_bias ? Ly.router_bias[q] : 0.0f);
+                else *sgate = 1.0f / (1.0f + expf(-v));
             }
         }
-        grid_barrier(p.ctl, nblocks, bar_idx++, to);
+        // the logits are published; while the other blocks finish theirs, warps 1..7 stream
+        // the shared expert's gate/up rows (it needs no routing: the extra expert slot of the
+        // DwarfStar MoE kernel) and warp 0 alone waits for the barrier, then takes the top-k.
+        // Pair i goes to block i % nblocks; its slot i / nblocks (mod 7) picks the warp:
+        // slots 0..3 are warps 4..7, which had no router row, slots 4..6 warps 1..3.
+        grid_arrive(p.ctl);
+        const unsigned bar1 = bar_idx++;
+        const int shslot = warp >= 4 ? warp - 4 : (warp > 0 ? warp + 3 : -1);
+        for (int i = shslot < 0 ? I : shslot * nblocks + blockIdx.x; i < I; i += 7 * nblocks) {
+            float xr[D1_XPL];
+            Row g, u;
+            ld_row<WT>(g, static_cast<const char*>(Ly.sh_gate) + size_t(i) * grow,
+                       PACKED ? Ly.sh_s_gate + size_t(i) * (H / 32) : nullptr, H, lane);
+            ld_row<WT>(u, static_cast<const char*>(Ly.sh_up) + size_t(i) * grow,
+                       PACKED ? Ly.sh_s_up + size_t(i) * (H / 32) : nullptr, H, lane);
+            mbar_wait(xbar, par, err, to);
+            load_x<WT, true>(reinterpret_cast<const uint16_t*>(smem + S.xs), H, lane, xr);
+            const float a = hsum2(dot_row<WT>(g, xr)), b = hsum2(dot_row<WT>(u, xr));
+            if (lane == 0) hsh[i] = silu_mul(a, b);
+        }
 
-        // Phase C's work comes in units (slot u, half hf of the block's rows): the shared
-        // expert's two units (warps 1 and 2, while warp 0 takes the top-k) and the routed
-        // 2 k units (unit = warp + 8 m, every unit of a warp has hf = warp & 1). Each warp
-        // accumulates its rows' weighted partials in registers.
-        constexpr int MU = (2 * D1_MAXK + D1_WARPS - 1) / D1_WARPS;  // routed units per warp, at most
+        // Phase C's work comes in units (slot u, half hf of the block's rows): 2 (k + 1)
+        // units, slots 0 .. k-1 the routed experts and slot k the shared one (unit = warp +
+        // 8 m, every unit of a warp has hf = warp & 1). Each warp accumulates its rows'
+        // weighted partials in registers.
+        constexpr int MU = (2 * (D1_MAXK + 1) + D1_WARPS - 1) / D1_WARPS;  // units per warp, at most
         const int half = (nrows + 1) / 2;
         const int ra = (warp & 1) * half, rn = nrows > 0 ? min(half, nrows - ra) : 0;
         float2 acc[D1_RB_MAX / 2];
-#pragma unroll
-        for (int r = 0; r < D1_RB_MAX / 2; ++r) acc[r] = make_float2(0.f, 0.f);
         // weighted row dots of one unit: acc[r] += wu * (row ra + r of slot u) . h
         auto unit_dots = [&](int u, float wu, const float (&hf32)[D1_HPL]) {
             mbar_wait(dbar + u, par, err, to);
@@ -213,12 +226,10 @@ __global__ void __launch_bounds__(D1_THREADS, 1) decode1_kernel(const __grid_con
             }
         };
         // ------------------------------------------------------------ phase B
-        // x in the layout of the expert weights
-        float xf[D1_XPL];
-        load_x<WT>(x, H, lane, xf);
         if (warp == 0) {
             // one warp per block takes the top-k of the logits (lane j < k: id and
             // renormalised weight of selection j) and shares it
+            grid_wait_warp(p.ctl, nblocks, bar1, to);
             int id = 0;
             float wv = 0.0f;
             if (Ly.given_ids) {
@@ -246,19 +257,14 @@ __global__ void __launch_bounds__(D1_THREADS, 1) decode1_kernel(const __grid_con
                     Ly.w[lane] = wv;
                 }
             }
-        } else if (warp <= 2 && nrows > 0) {
-            // meanwhile warps 1 and 2 take phase C's two units of the shared expert (its h
-            // and its down rows are ready: phase A made them)
-            float hh[D1_HPL];
-            const float4* hv = reinterpret_cast<const float4*>(hsh + lane * D1_HPL);
-#pragma unroll
-            for (int i = 0; i < D1_HPL / 4; ++i) {
-                const float4 v = __ldcg(hv + i);
-                hh[4 * i] = v.x; hh[4 * i + 1] = v.y; hh[4 * i + 2] = v.z; hh[4 * i + 3] = v.w;
-            }
-            unit_dots(k, __ldcg(sgate), hh);
         }
         __syncthreads();
+#pragma unroll
+        for (int r = 0; r < D1_RB_MAX / 2; ++r) acc[r] = make_float2(0.f, 0.f);
+        // x in the layout of the expert weights (from the shared copy: no memory latency)
+        float xf[D1_XPL];
+        mbar_wait(xbar, par, err, to);
+        load_x<WT, true>(reinterpret_cast<const uint16_t*>(smem + S.xs), H, lane, xf);
         const int sel_id = lane < k ? s_sel_slot[lane] : 0;  // stack index of selection j
         const float sel_w = lane < k ? s_sel_w[lane] : 0.0f;
         if (warp == 0 && nrows > 0) {
@@ -319,18 +325,20 @@ __global__ void __launch_bounds__(D1_THREADS, 1) decode1_kernel(const __grid_con
         }
         if (nrows > 0) {
             if (threadIdx.x == 0) {
-                // the routed h rows (written by every block before the barrier) into shared
-                // memory with one bulk copy
+                // the routed and the shared h rows (written by every block before the
+                // barrier) into shared memory, two bulk copies
                 fence_proxy_async_global();
                 fence_proxy_async_smem();
-                mbar_arrive_expect_tx(hbar, uint32_t(4 * k * I));
+                mbar_arrive_expect_tx(hbar, uint32_t(4 * (k + 1) * I));
                 bulk_g2s(smem + S.hbuf, p.hrt, uint32_t(4 * k * I), hbar);
+                bulk_g2s(smem + S.hbuf + 4 * k * I, hsh, uint32_t(4 * I), hbar);
             }
             mbar_wait(hbar, par, err, to);
+            const float wsh = __ldcg(sgate);
 #pragma unroll 1
             for (int m = 0; m < MU; ++m) {
                 const int unit = warp + D1_WARPS * m;
-                if (unit < 2 * k) {
+                if (unit < 2 * (k + 1)) {
                     const int u = unit >> 1;
                     float hh[D1_HPL];
                     const float4* hv = reinterpret_cast<const float4*>(hbuf + size_t(u) * I + lane * D1_HPL);
@@ -339,7 +347,8 @@ __global__ void __launch_bounds__(D1_THREADS, 1) decode1_kernel(const __grid_con
                         const float4 v = hv[i];
                         hh[4 * i] = v.x; hh[4 * i + 1] = v.y; hh[4 * i + 2] = v.z; hh[4 * i + 3] = v.w;
                     }
-                    unit_dots(u, __shfl_sync(FULL, sel_w, u), hh);
+                    const float wr = __shfl_sync(FULL, sel_w, u < k ? u : 0);
+                    unit_dots(u, u < k ? wr : wsh, hh);
                 }
             }
         }
@@ -390,7 +399,7 @@ redmoe_status d1_launch(const redmoe_layer* sh, const DecLayer* layers, int n_la
     if (!get_dev_info(&di)) return REDMOE_ERR_CUDA;
     const int RB = (sh->hidden + di.sm_count - 1) / di.sm_count;
     if (RB > D1_RB_MAX) return REDMOE_ERR_UNSUPPORTED;
-    const D1Smem S = d1_smem(WT, sh->top_k, sh->inter, RB);
+    const D1Smem S = d1_smem(WT, sh->top_k, sh->inter, RB, sh->hidden);
     if (S.total > di.max_smem_optin) return REDMOE_ERR_UNSUPPORTED;
     auto kern = decode1_kernel<WT, NL>;
     const int per_sm = d1_blocks_per_sm(reinterpret_cast<const void*>(kern), S.total);

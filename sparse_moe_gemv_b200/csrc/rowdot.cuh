@@ -31,7 +31,8 @@ template <> struct ChunkElems<DT_INT2> { static constexpr int n = 64; };
 //   bf16 rows: chunk c = lane + 32 j (j < H / 256) covers elements 8c .. 8c + 7 -> xf[8j + m]
 //   int4 rows: chunk c = lane + 32 j (j < H / 1024) covers elements 32c .. 32c + 31 -> xf[32j + m]
 //   int2 rows: chunk c = lane (H = 2048) covers elements 64c .. 64c + 63 -> xf[m]
-template <int W>
+// SM: x is a copy in shared memory (plain loads) rather than in global memory.
+template <int W, bool SM = false>
 __device__ __forceinline__ void load_x(const uint16_t* x, int H, int lane, float (&xf)[D1_XPL]) {
     constexpr int PER = ChunkElems<W>::n;  // elements per chunk
     constexpr int NJ = D1_XPL / PER;
@@ -42,8 +43,8 @@ __device__ __forceinline__ void load_x(const uint16_t* x, int H, int lane, float
 #pragma unroll
         for (int q = 0; q < PER / 8; ++q) {
             const bool ok = (c * PER + q * 8) < H;
-            v[j * (PER / 8) + q] = ok ? __ldg(reinterpret_cast<const uint4*>(x + size_t(c) * PER + q * 8))
-                                      : make_uint4(0u, 0u, 0u, 0u);
+            const uint4* px = reinterpret_cast<const uint4*>(x + size_t(c) * PER + q * 8);
+            v[j * (PER / 8) + q] = ok ? (SM ? *px : __ldg(px)) : make_uint4(0u, 0u, 0u, 0u);
         }
     }
 #pragma unroll

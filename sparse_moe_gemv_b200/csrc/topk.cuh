@@ -82,14 +82,13 @@ __device__ __forceinline__ void warp_topk_keys(int E, int k, const uint32_t* key
 // token's logit range (max - min over the E logits), ties to the lower id; the weights are
 // the softmax of the unbiased logits over the selected experts (the bias changes which
 // experts run, not how their outputs are mixed). Lane j < k ends with (id_j, w_j).
+// The same from logits already in registers: z[i] of lane L is expert i * 32 + L (any
+// value past E; it is not selected).
 template <int EPL>
-__device__ __forceinline__ void warp_route(const float* logits, int E, int k, const uint8_t* cached, float lambda,
-                                           int& out_id, float& out_w) {
+__device__ __forceinline__ void warp_route_z(const float (&z)[EPL], int E, int k, const uint8_t* cached, float lambda,
+                                             int& out_id, float& out_w) {
     const int lane = threadIdx.x & 31;
-    float z[EPL];
     uint32_t key[EPL];
-#pragma unroll
-    for (int i = 0; i < EPL; ++i) z[i] = (i * 32 + lane < E) ? __ldcg(logits + i * 32 + lane) : 0.0f;
     if (cached == nullptr) {
 #pragma unroll
         for (int i = 0; i < EPL; ++i) key[i] = (i * 32 + lane < E) ? order_key(z[i]) : 0u;
@@ -113,13 +112,29 @@ __device__ __forceinline__ void warp_route(const float* logits, int E, int k, co
     }
     float wb;
     warp_topk_core<EPL>(key, k, out_id, wb);
-    // weights from the unbiased logits of the selection
-    const float zj = lane < k ? __ldcg(logits + out_id) : -INFINITY;
+    // weights from the unbiased logits of the selection: lane j fetches z of its id from
+    // the lane that holds it
+    float zj = -INFINITY;
+#pragma unroll
+    for (int i = 0; i < EPL; ++i) {
+        const float v = __shfl_sync(FULL, z[i], out_id & 31);
+        if (lane < k && (out_id >> 5) == i) zj = v;
+    }
     float m = zj;
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(FULL, m, o));
     const float ex = lane < k ? expf(zj - m) : 0.0f;
     out_w = ex / warp_sum(ex);
+}
+
+template <int EPL>
+__device__ __forceinline__ void warp_route(const float* logits, int E, int k, const uint8_t* cached, float lambda,
+                                           int& out_id, float& out_w) {
+    const int lane = threadIdx.x & 31;
+    float z[EPL];
+#pragma unroll
+    for (int i = 0; i < EPL; ++i) z[i] = (i * 32 + lane < E) ? __ldcg(logits + i * 32 + lane) : 0.0f;
+    warp_route_z<EPL>(z, E, k, cached, lambda, out_id, out_w);
 }
 
 // warp_route with EPL chosen from E.

@@ -6,8 +6,9 @@ import pytest
 import torch
 
 import moe_inputs as mi
+import oracle
 import sparse_moe_gemv_b200 as smg
-from parity import assert_layer_parity, tolerances
+from parity import assert_layer_parity, host_routing_layer, reference, tolerances
 
 pytestmark = pytest.mark.gpu
 
@@ -73,6 +74,54 @@ def test_qwen_int2(gpu_lib):
         out, ids, w, _, _ = _run(gpu_lib, shape, L, x)
         ot, wt = tolerances(shape)
         assert_layer_parity(shape, L, x, out, ids, w, ot, wt, f"int2 seed={seed}")
+
+
+@pytest.mark.parametrize("case", ["ties_in_topk", "ties_at_boundary", "all_equal"])
+def test_router_ties_one_row(gpu_lib, case):
+    """Exactly equal logits (duplicated router rows) go to the lower expert id first, in
+    the selection and in its order: inside the top-k, across the k-th place, and with all
+    E logits equal (every key reaches the selection threshold, so the one-row kernel takes
+    its round-by-round fallback)."""
+    shape = QWEN
+    L = _dev_layer(shape, 1100)
+    x = mi.make_x(shape, 1, 1100, "cuda")
+    out, ids, w, _, _ = _run(gpu_lib, shape, L, x)
+    top = ids[0].tolist()
+    R = L["router_w"]
+    if case == "ties_in_topk":
+        # the 3rd-ranked expert's row copied to two lower and two higher ids
+        src = top[2]
+        for e in (0, 1, 510, 511):
+            if e not in top:
+                R[e] = R[src]
+    elif case == "ties_at_boundary":
+        # the 10th-ranked expert's row copied to four other experts: a 5-way tie that only
+        # the lowest ids survive
+        src = top[9]
+        for e in (3, 77, 300, 509):
+            if e not in top:
+                R[e] = R[src]
+    else:
+        R[:] = R[0]
+    out, ids, w, _, _ = _run(gpu_lib, shape, L, x)
+    ot, wt = tolerances(shape)
+    if case != "all_equal":
+        ref = reference(shape, L, x)
+        assert ids[0].tolist() == [int(e) for e in ref["ids"][0]], (ids[0].tolist(), ref["ids"][0])
+        assert_layer_parity(shape, L, x, out, ids, w, ot, wt, f"ties {case}")
+        return
+    # every expert ties: the oracle's own routing (no near-tie enumeration, which would
+    # list every k-subset of the 512) and its outputs for that routing
+    xn = mi.to_numpy(x)
+    r = oracle.router(host_routing_layer(L), shape, xn)
+    assert r["ids"][0].tolist() == list(range(shape.k))
+    assert ids[0].tolist() == list(range(shape.k))
+    assert np.allclose(w[0].cpu().numpy(), 1.0 / shape.k, atol=1e-6)
+    lay_e = mi.layer_to_numpy(L, experts=list(range(shape.k)))
+    ref_out = oracle.experts(lay_e, shape, xn, r["ids"], r["w"], r["s"])
+    rms = float(np.sqrt(np.mean(ref_out ** 2)))
+    err = float(np.max(np.abs(out.cpu().numpy().astype(np.float64) - ref_out)))
+    assert err <= ot * rms, (err, rms)
 
 
 def test_int2_beyond_one_row_is_unsupported(gpu_lib):
