@@ -243,6 +243,21 @@ __device__ __forceinline__ void grid_wait_warp(Control* ctl, unsigned nblocks, u
     __syncwarp();
 }
 
+// The block has passed the launch's last wait on the barrier counters: count it out; the
+// last block out resets the counters for the next launch. Thread 0 calls it right after
+// the final grid_barrier / grid_wait, so the two atomic round trips of the reset overlap
+// the rest of the launch instead of lengthening its tail. A launch uses either this or
+// grid_exit.
+__device__ __forceinline__ void grid_release(Control* ctl, unsigned nblocks) {
+    if (threadIdx.x == 0) {
+        const unsigned done = atomicAdd(&ctl->bar_gen, 1u);
+        if (done == nblocks - 1u) {
+            atomicExch(&ctl->bar_count, 0u);
+            atomicExch(&ctl->bar_gen, 0u);
+        }
+    }
+}
+
 // End of a launch that used grid_barrier: the last block out resets the counters.
 __device__ __forceinline__ void grid_exit(Control* ctl, unsigned nblocks) {
     __syncthreads();

@@ -577,6 +577,7 @@ __global__ void __launch_bounds__(THREADS, 1) decode_kernel(const __grid_constan
         ring.set_depth(NS);  // drained: phase C keeps the h buffer for h
         while (has_rows && !ring.full() && cj < jobsC) { ring.issue(segC(cj), lane); cj += gpc; }
         grid_wait(p.ctl, nblocks, bar_idx++, to);
+        if (l + 1 == p.n_layers) grid_release(p.ctl, nblocks);  // the launch's last barrier
 
         // ---------------------------------------------------------- phase C
         if (threadIdx.x == 0) {
@@ -666,7 +667,6 @@ __global__ void __launch_bounds__(THREADS, 1) decode_kernel(const __grid_constan
         }
         if (l + 1 < p.n_layers) grid_barrier(p.ctl, nblocks, bar_idx++, to);
     }
-    grid_exit(p.ctl, nblocks);
 }
 
 // Down rows per phase-C stage: as many as fit one stage (with their int4 scales), at most

@@ -312,6 +312,7 @@ __global__ void __launch_bounds__(D1_THREADS, 1) decode1_kernel(const __grid_con
 
         // ------------------------------------------------------------ phase C
         grid_barrier(p.ctl, nblocks, bar_idx++, to);
+        if (l + 1 == p.n_layers) grid_release(p.ctl, nblocks);  // the launch's last barrier
         if (l + 1 < p.n_layers && threadIdx.x < 32) {
             // L2 prefetch of the next layer's router rows and shared gate/up rows (the rows
             // this block streams first in that layer)
@@ -367,7 +368,6 @@ __global__ void __launch_bounds__(D1_THREADS, 1) decode1_kernel(const __grid_con
         }
         if (l + 1 < p.n_layers) grid_barrier(p.ctl, nblocks, bar_idx++, to);
     }
-    grid_exit(p.ctl, nblocks);
 }
 
 int d1_blocks_per_sm(const void* kern, int smem) {

@@ -363,6 +363,7 @@ __global__ void __launch_bounds__(D1_THREADS, 1) decodefr_kernel(const __grid_co
             }
         }
         grid_barrier(p.ctl, nblocks, bar_idx++, to);
+        if (l + 1 == p.n_layers) grid_release(p.ctl, nblocks);  // the launch's last barrier
 
         // ------------------------------------------------------------ phase C
         if (l + 1 < p.n_layers && threadIdx.x < 32) {
@@ -434,7 +435,6 @@ __global__ void __launch_bounds__(D1_THREADS, 1) decodefr_kernel(const __grid_co
         }
         if (l + 1 < p.n_layers) grid_barrier(p.ctl, nblocks, bar_idx++, to);
     }
-    grid_exit(p.ctl, nblocks);
 }
 
 int fr_blocks_per_sm(const void* kern, int smem) {

@@ -177,6 +177,7 @@ __global__ void __launch_bounds__(RT_THREADS, 1) route_kernel(const __grid_const
         if (lane == 0) p.counts[e] = carry;
     }
     grid_barrier(p.ctl, nb, 1, p.timeout_ns);
+    grid_release(p.ctl, nb);  // the launch's last barrier
 
     // ------------------------------------------------------------------ phase 3
     for (int e = threadIdx.x; e < E; e += RT_THREADS) tmp[e] = __ldcg(p.counts + e);
@@ -250,7 +251,6 @@ __global__ void __launch_bounds__(RT_THREADS, 1) route_kernel(const __grid_const
             }
         }
     }
-    grid_exit(p.ctl, nb);
 }
 
 int route_smem_bytes(int E, int tpb, int k) { return 4 * (3 * E + 1 + 32 + 2 * tpb * k); }
