@@ -503,15 +503,24 @@ def gpu_arm(args, wl, world, rank, local, B=None, name=None):
     achieved = bytes_per_launch / launch_s / 1e9
     key = name or args.workload
     if T > 4:
-        # batched path: four kernels per step; the roofline is the tensor-core one of the layer
+        # batched path: four kernels per step. Its roofline is the binding one of two: the
+        # step's algorithmic bytes (every touched expert's weights once, x, out) at the HBM
+        # peak, and its FLOPs at the bf16 tensor peak. With a few tokens per expert the
+        # weights dominate and the HBM time is the larger.
         flops = layer_flops(shape, T)
         step_s = el_ms / 1e3 / K
         tfl = flops / step_s / 1e12
-        roof = {"bound": "tensor", "achieved": tfl, "peak": bf16, "unit": "TFLOP/s", "frac": tfl / bf16,
-                "traffic": profile_traffic(key), "kernel": wl["kernel"], "flops_per_step": flops,
-                "weight_bytes_per_step": bytes_per_launch, "hbm_gbs_of_weights": bytes_per_launch / step_s / 1e9,
-                "hbm_frac_of_weights": bytes_per_launch / step_s / 1e9 / hbm,
-                "peak_source": f"{src} (MEASURED_PEAKS.json bf16_tflops, burst)"}
+        gbs = bytes_per_launch / step_s / 1e9
+        t_hbm, t_tc = bytes_per_launch / (hbm * 1e9), flops / (bf16 * 1e12)
+        both = {"traffic": profile_traffic(key), "kernel": wl["kernel"], "flops_per_step": flops,
+                "bytes_per_step": bytes_per_launch, "hbm_floor_us": t_hbm * 1e6, "tensor_floor_us": t_tc * 1e6,
+                "tensor_tflops": tfl, "tensor_frac": tfl / bf16, "hbm_gbs": gbs, "hbm_frac": gbs / hbm}
+        if t_hbm >= t_tc:
+            roof = {"bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s", "frac": gbs / hbm, **both,
+                    "peak_source": f"{src} (MEASURED_PEAKS.json hbm_gbs)" if src == "measured" else "fallback"}
+        else:
+            roof = {"bound": "tensor", "achieved": tfl, "peak": bf16, "unit": "TFLOP/s", "frac": tfl / bf16, **both,
+                    "peak_source": f"{src} (MEASURED_PEAKS.json bf16_tflops, burst)"}
         launches = K * 4
     else:
         roof = {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
