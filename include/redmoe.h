@@ -194,6 +194,23 @@ size_t redmoe_expert_cache_slot_bytes(const redmoe_layer *L);
 /* Empty the cache on `stream`: every slot free, hotness and counters zero. */
 redmoe_status redmoe_expert_cache_init(const redmoe_layer *L, redmoe_expert_cache *cache, void *stream);
 
+/* redmoe_forward with the activations and results in HOST memory: the call a host
+ * program makes per step. x_host [T, H] (L->x_dtype) is copied into the workspace's
+ * device staging area with one cudaMemcpyAsync (any host memory; pinned keeps it
+ * asynchronous). At decode sizes (T <= 4), when out_host, ids_host and w_host are pinned
+ * (page-locked) host memory, the kernel stores the results straight into them through
+ * their device mapping, so no copy back is enqueued; otherwise (T > 4, or pageable
+ * outputs) the results go to device staging and three cudaMemcpyAsync bring them back.
+ * Either way the results are in host memory once `stream` has reached the end of the
+ * call: synchronise it before reading them. Same layouts, alignment rules (16 bytes for
+ * x and out, 4 for ids and w) and statuses as redmoe_forward; the workspace must hold
+ * redmoe_workspace_bytes_host(L, T) bytes (the forward's workspace, then the staging).
+ * The arithmetic is redmoe_forward's; the pages have no separate counterpart. */
+size_t redmoe_workspace_bytes_host(const redmoe_layer *L, int32_t T);
+redmoe_status redmoe_forward_host(const redmoe_layer *L, const void *x_host, int32_t T, float *out_host,
+                                  int32_t *ids_host, float *w_host, void *workspace, size_t workspace_bytes,
+                                  void *stream);
+
 /* redmoe_forward for one token row (T = 1) whose routed expert stacks (w_gate, w_up,
  * w_down and their scales) may live in pinned host memory that the device can read
  * (cudaHostAlloc / cudaHostRegister, e.g. torch pin_memory); router, shared gate and

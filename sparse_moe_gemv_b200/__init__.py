@@ -32,7 +32,8 @@ SYMBOLS = ("redmoe_abi_version", "redmoe_status_string", "redmoe_workspace_bytes
            "redmoe_forward", "redmoe_router", "redmoe_route_build", "redmoe_forward_stack",
            "redmoe_check_timeout", "redmoe_forward_noalloc", "redmoe_selftest_wait_limit",
            "redmoe_fill_shared_memory", "redmoe_forward_cached", "redmoe_expert_cache_slot_bytes",
-           "redmoe_expert_cache_init", "redmoe_forward_host_experts", "redmoe_expert_cache_prefetch")
+           "redmoe_expert_cache_init", "redmoe_forward_host_experts", "redmoe_expert_cache_prefetch",
+           "redmoe_workspace_bytes_host", "redmoe_forward_host")
 
 _lock = threading.Lock()
 _lib = None
@@ -112,6 +113,10 @@ def load():
         lib.redmoe_expert_cache_prefetch.argtypes = [P, P, P, i32, P, sz, P]
         lib.redmoe_fill_shared_memory.restype = i32
         lib.redmoe_fill_shared_memory.argtypes = [C.c_uint32, P]
+        lib.redmoe_workspace_bytes_host.restype = sz
+        lib.redmoe_workspace_bytes_host.argtypes = [P, i32]
+        lib.redmoe_forward_host.restype = i32
+        lib.redmoe_forward_host.argtypes = [P, P, i32, P, P, P, P, sz, P]
         if lib.redmoe_abi_version() != ABI_VERSION:
             raise RuntimeError("libredmoe.so ABI version mismatch")
         _lib = lib
@@ -207,6 +212,29 @@ def redmoe_forward(layer: Layer, x: torch.Tensor, out: torch.Tensor, topk_ids: t
                             _ptr(workspace), workspace.numel() * workspace.element_size(),
                             None if dbg_s is None else C.byref(dbg_s), _stream(stream))
     _check(st, "redmoe_forward")
+
+
+def redmoe_workspace_bytes_host(layer: Layer, T: int) -> int:
+    return int(load().redmoe_workspace_bytes_host(layer.ref, int(T)))
+
+
+def new_workspace_host(layer: Layer, T: int, device=None) -> torch.Tensor:
+    """A zeroed workspace tensor of redmoe_workspace_bytes_host(layer, T) bytes."""
+    n = redmoe_workspace_bytes_host(layer, T)
+    if n == 0:
+        raise ValueError("invalid layer or token count")
+    return torch.zeros(n, dtype=torch.uint8, device=device or "cuda")
+
+
+def redmoe_forward_host(layer: Layer, x_host: torch.Tensor, out_host: torch.Tensor, ids_host: torch.Tensor,
+                        w_host: torch.Tensor, workspace: torch.Tensor, stream=None) -> None:
+    """redmoe_forward with x and the results in host memory (pinned for asynchronous
+    copies, and for results stored straight from the kernel at T <= 4). The results are
+    valid once `stream` has been synchronised."""
+    T = x_host.shape[0]
+    st = load().redmoe_forward_host(layer.ref, _ptr(x_host), int(T), _ptr(out_host), _ptr(ids_host), _ptr(w_host),
+                                    _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream))
+    _check(st, "redmoe_forward_host")
 
 
 def redmoe_forward_cached(layer: Layer, x: torch.Tensor, out: torch.Tensor, topk_ids: torch.Tensor,

@@ -200,6 +200,96 @@ redmoe_status redmoe_forward(const redmoe_layer* L, const void* x, int32_t T, fl
     return st;
 }
 
+namespace {
+
+// Device staging of redmoe_forward_host, after the forward's own workspace: x, then out,
+// ids and w (each 256-byte aligned).
+struct HostStage {
+    size_t x, out, ids, w, total;
+};
+HostStage host_stage_layout(const redmoe_layer* L, int T) {
+    HostStage h;
+    const size_t xb = L->x_dtype == DT_F32 ? 4 : 2;
+    size_t o = ws_bytes(L, T);
+    h.x = o; o = align256(o + xb * T * L->hidden);
+    h.out = o; o = align256(o + 4ull * T * L->hidden);
+    h.ids = o; o = align256(o + 4ull * T * L->top_k);
+    h.w = o; o = align256(o + 4ull * T * L->top_k);
+    h.total = o;
+    return h;
+}
+
+// The device mapping of pinned host memory (or the pointer itself for device memory);
+// null for memory the device cannot write (pageable host memory).
+void* writable_view(void* p) {
+    cudaPointerAttributes a;
+    if (cudaPointerGetAttributes(&a, p) != cudaSuccess) {
+        cudaGetLastError();
+        return nullptr;
+    }
+    if (a.type == cudaMemoryTypeDevice || a.type == cudaMemoryTypeManaged) return p;
+    if (a.type == cudaMemoryTypeHost) return a.devicePointer;
+    return nullptr;
+}
+
+}  // namespace
+
+size_t redmoe_workspace_bytes_host(const redmoe_layer* L, int32_t T) {
+    if (T < 0 || check_layer(L) == REDMOE_ERR_INVALID_ARG || !L) return 0;
+    return host_stage_layout(L, T).total;
+}
+
+redmoe_status redmoe_forward_host(const redmoe_layer* L, const void* x_host, int32_t T, float* out_host,
+                                  int32_t* ids_host, float* w_host, void* workspace, size_t workspace_bytes,
+                                  void* stream) {
+    redmoe_status st = check_layer(L);
+    if (st != REDMOE_OK) return st;
+    if (T < 0) return REDMOE_ERR_INVALID_ARG;
+    if (T == 0) return REDMOE_OK;
+    if (!x_host || !out_host || !ids_host || !w_host) return REDMOE_ERR_INVALID_ARG;
+    if (!aligned(x_host, 16) || !aligned(out_host, 16) || !aligned(ids_host, 4) || !aligned(w_host, 4))
+        return REDMOE_ERR_INVALID_ARG;
+    if (!workspace || !aligned(workspace, 256)) return REDMOE_ERR_WORKSPACE;
+    const HostStage h = host_stage_layout(L, T);
+    if (workspace_bytes < h.total) return REDMOE_ERR_WORKSPACE;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    char* base = static_cast<char*>(workspace);
+    if (T == 1 && decode1_shape_ok(L)) {
+        // one token row with every buffer pinned: the kernel reads x over the link once
+        // (block 0 stages it in the workspace) and stores the results straight back, so no
+        // copy is enqueued at all
+        const void* xv = writable_view(const_cast<void*>(x_host));
+        float* o = static_cast<float*>(writable_view(out_host));
+        int32_t* i = static_cast<int32_t*>(writable_view(ids_host));
+        float* w = static_cast<float*>(writable_view(w_host));
+        if (xv && o && i && w) {
+            const DecLayer d = dec_layer(L, xv, o, i, w);
+            return launch_decode1_host_x(L, &d, workspace, base + h.x, s);
+        }
+    }
+    const size_t xbytes = (L->x_dtype == DT_F32 ? 4ull : 2ull) * T * L->hidden;
+    if (cudaMemcpyAsync(base + h.x, x_host, xbytes, cudaMemcpyDefault, s) != cudaSuccess) return REDMOE_ERR_CUDA;
+    if (T <= DECODE_MAX_T) {
+        // the decode kernels store each result once: straight into mapped host memory
+        float* o = static_cast<float*>(writable_view(out_host));
+        int32_t* i = static_cast<int32_t*>(writable_view(ids_host));
+        float* w = static_cast<float*>(writable_view(w_host));
+        if (o && i && w)
+            return redmoe_forward(L, base + h.x, T, o, i, w, workspace, workspace_bytes, nullptr, stream);
+    }
+    float* o = reinterpret_cast<float*>(base + h.out);
+    int32_t* i = reinterpret_cast<int32_t*>(base + h.ids);
+    float* w = reinterpret_cast<float*>(base + h.w);
+    if ((st = redmoe_forward(L, base + h.x, T, o, i, w, workspace, workspace_bytes, nullptr, stream)) != REDMOE_OK)
+        return st;
+    const size_t kb = 4ull * T * L->top_k;
+    if (cudaMemcpyAsync(out_host, o, 4ull * T * L->hidden, cudaMemcpyDefault, s) != cudaSuccess ||
+        cudaMemcpyAsync(ids_host, i, kb, cudaMemcpyDefault, s) != cudaSuccess ||
+        cudaMemcpyAsync(w_host, w, kb, cudaMemcpyDefault, s) != cudaSuccess)
+        return REDMOE_ERR_CUDA;
+    return REDMOE_OK;
+}
+
 redmoe_status redmoe_forward_cached(const redmoe_layer* L, const void* x, int32_t T, float* out, int32_t* topk_ids,
                                     float* topk_w, const uint8_t* cached, float lambda, void* workspace,
                                     size_t workspace_bytes, void* stream) {

@@ -18,7 +18,8 @@ struct Control {
     unsigned bar_count;   // grid-barrier arrivals since the launch began
     unsigned bar_gen;     // blocks that have finished the launch (grid_exit)
     int err;              // ERRBIT_* set by any kernel that gave up waiting
-    unsigned pad[61];
+    unsigned x_ready;     // one-row kernel: x copied from host memory into the workspace
+    unsigned pad[60];
 };
 static_assert(sizeof(Control) == 256, "control block is 256 bytes");
 
@@ -244,16 +245,17 @@ __device__ __forceinline__ void grid_wait_warp(Control* ctl, unsigned nblocks, u
 }
 
 // The block has passed the launch's last wait on the barrier counters: count it out; the
-// last block out resets the counters for the next launch. Thread 0 calls it right after
-// the final grid_barrier / grid_wait, so the two atomic round trips of the reset overlap
-// the rest of the launch instead of lengthening its tail. A launch uses either this or
-// grid_exit.
+// last block out resets the counters (and the x-ready flag) for the next launch. Thread 0
+// calls it right after the final grid_barrier / grid_wait, so the atomic round trips of
+// the reset overlap the rest of the launch instead of lengthening its tail. A launch uses
+// either this or grid_exit.
 __device__ __forceinline__ void grid_release(Control* ctl, unsigned nblocks) {
     if (threadIdx.x == 0) {
         const unsigned done = atomicAdd(&ctl->bar_gen, 1u);
         if (done == nblocks - 1u) {
             atomicExch(&ctl->bar_count, 0u);
             atomicExch(&ctl->bar_gen, 0u);
+            atomicExch(&ctl->x_ready, 0u);
         }
     }
 }

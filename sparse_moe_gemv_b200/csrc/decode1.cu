@@ -80,6 +80,9 @@ struct D1Params {
     float* hrt;     // [k, I]
     uint64_t timeout_ns;
     CacheBias cb;
+    // non-null: layer 0's x is pinned host memory (its device mapping in L[0].x); block 0
+    // copies it here and raises Control::x_ready, and every block reads it from here
+    uint16_t* xstage;
     DecLayer L[NL];
 };
 
@@ -136,11 +139,49 @@ __global__ void __launch_bounds__(D1_THREADS, 1) decode1_kernel(const __grid_con
         const uint32_t par = uint32_t(l & 1);
 
         // ------------------------------------------------------------ phase A
-        if (threadIdx.x == 0) {
-            fence_proxy_async_smem();  // the previous layer's reads of dreg and xs come first
+        const bool xremote = p.xstage != nullptr && l == 0;
+        if (xremote && blockIdx.x == 0 && warp >= 4) {
+            // x from host memory: warps 4..7 of block 0 (no router row) read it once over the
+            // link with cache-volatile loads (the host rewrites it between calls), every load
+            // of a lane issued before its first store so that the copy costs one link round
+            // trip, write it to the workspace and count themselves on x_ready
+            constexpr int PER = D1_XPL / 32;  // 16-byte chunks per lane: a quarter of x per warp
+            const uint4* src = reinterpret_cast<const uint4*>(x);
+            uint4* dst = reinterpret_cast<uint4*>(p.xstage);
+            const int c0 = (warp - 4) * 32 * PER + lane;
+            uint4 v[PER];
+#pragma unroll
+            for (int j = 0; j < PER; ++j)
+                if (c0 + 32 * j < H / 8) v[j] = __ldcv(src + c0 + 32 * j);
+#pragma unroll
+            for (int j = 0; j < PER; ++j)
+                if (c0 + 32 * j < H / 8) dst[c0 + 32 * j] = v[j];
+            __threadfence();
+            __syncwarp();
+            if (lane == 0) asm volatile("red.release.gpu.global.add.u32 [%0], 1;" :: "l"(&p.ctl->x_ready) : "memory");
+        }
+        if (threadIdx.x == (xremote ? 32 * (D1_WARPS - 1) : 0)) {
+            // (with x in host memory an idle warp's lane waits for it, so that warp 0's
+            // router row is not held up)
+            const void* xsrc = x;
+            if (xremote) {
+                const uint64_t t0 = globaltimer_ns();
+                for (uint32_t spins = 0; ld_acquire_gpu(&p.ctl->x_ready) < 4u; ++spins) {
+                    if ((spins & 63u) == 63u && (globaltimer_ns() - t0 > to || spins > (1u << 26))) {
+                        atomicOr(err, ERRBIT_TIMEOUT);
+                        break;
+                    }
+                }
+                fence_proxy_async_global();  // generic stores of block 0, read by the bulk copy
+                xsrc = p.xstage;
+            }
+            fence_proxy_async_smem();  // the previous layer's reads of xs come first
             mbar_arrive_expect_tx(xbar, uint32_t(2 * H));
-            bulk_g2s(smem + S.xs, x, uint32_t(2 * H), xbar);
-            if (nrows > 0) issue_down(k, Ly.sh_down, Ly.sh_s_down);
+            bulk_g2s(smem + S.xs, xsrc, uint32_t(2 * H), xbar);
+        }
+        if (threadIdx.x == 0 && nrows > 0) {
+            fence_proxy_async_smem();  // the previous layer's reads of dreg come first
+            issue_down(k, Ly.sh_down, Ly.sh_s_down);
         }
         // job q < E: router row q; q == E: shared-gate row. Warp w of block b takes
         // q = w * nblocks + b: the jobs go to the low warps of every block. Only these rows
@@ -394,7 +435,7 @@ int d1_blocks_per_sm(const void* kern, int smem) {
 
 template <int WT, int NL>
 redmoe_status d1_launch(const redmoe_layer* sh, const DecLayer* layers, int n_layers, void* ws, cudaStream_t stream,
-                        CacheBias cb) {
+                        CacheBias cb, void* xstage = nullptr) {
     DevInfo di;
     if (!get_dev_info(&di)) return REDMOE_ERR_CUDA;
     const int RB = (sh->hidden + di.sm_count - 1) / di.sm_count;
@@ -421,6 +462,7 @@ redmoe_status d1_launch(const redmoe_layer* sh, const DecLayer* layers, int n_la
     q.hrt = reinterpret_cast<float*>(base + L.hrt);
     q.timeout_ns = BARRIER_TIMEOUT_NS;
     q.cb = cb;
+    q.xstage = static_cast<uint16_t*>(xstage);
     for (int i = 0; i < n_layers; ++i) q.L[i] = layers[i];
 
     cudaLaunchConfig_t cfg = {};
@@ -440,10 +482,10 @@ redmoe_status d1_launch(const redmoe_layer* sh, const DecLayer* layers, int n_la
 
 template <int WT>
 redmoe_status d1_launch_all(const redmoe_layer* sh, const DecLayer* layers, int n_layers, void* ws, cudaStream_t stream,
-                            int* launches, CacheBias cb) {
+                            int* launches, CacheBias cb, void* xstage = nullptr) {
     redmoe_status st = REDMOE_OK;
     if (n_layers == 1) {
-        st = d1_launch<WT, 1>(sh, layers, 1, ws, stream, cb);
+        st = d1_launch<WT, 1>(sh, layers, 1, ws, stream, cb, xstage);
         if (st == REDMOE_OK && launches) *launches += 1;
         return st;
     }
@@ -475,6 +517,14 @@ redmoe_status launch_decode1(const redmoe_layer* sh, const DecLayer* layers, int
     if (sh->expert_dtype == DT_INT4) return d1_launch_all<DT_INT4>(sh, layers, n_layers, ws, stream, launches, cb);
     if (sh->expert_dtype == DT_INT2) return d1_launch_all<DT_INT2>(sh, layers, n_layers, ws, stream, launches, cb);
     return d1_launch_all<DT_BF16>(sh, layers, n_layers, ws, stream, launches, cb);
+}
+
+redmoe_status launch_decode1_host_x(const redmoe_layer* sh, const DecLayer* layer, void* ws, void* xstage,
+                                    cudaStream_t stream) {
+    const CacheBias cb{nullptr, 0.0f};
+    if (sh->expert_dtype == DT_INT4) return d1_launch_all<DT_INT4>(sh, layer, 1, ws, stream, nullptr, cb, xstage);
+    if (sh->expert_dtype == DT_INT2) return d1_launch_all<DT_INT2>(sh, layer, 1, ws, stream, nullptr, cb, xstage);
+    return d1_launch_all<DT_BF16>(sh, layer, 1, ws, stream, nullptr, cb, xstage);
 }
 
 }  // namespace redmoe

@@ -102,6 +102,34 @@ def test_forward_rejects_bad_call_arguments(lib):
     assert _fwd(lib, L, T=0) == OK
 
 
+def test_forward_host_checks_before_touching_cuda(lib):
+    """The host-buffer forward: its workspace holds the forward's plus the staging, and bad
+    arguments are rejected before any copy is enqueued."""
+    L = _layer()
+    for T in (1, 4, 5, 2048):
+        n, nh = lib.redmoe_workspace_bytes(C.byref(L), T), lib.redmoe_workspace_bytes_host(C.byref(L), T)
+        # staging: x (bf16) + out (fp32) + ids + w, each 256-aligned
+        assert nh % 256 == 0 and nh >= n + T * 2048 * 2 + T * 2048 * 4 + 2 * T * 10 * 4
+    assert lib.redmoe_workspace_bytes_host(C.byref(L), -1) == 0
+    assert lib.redmoe_workspace_bytes_host(None, 1) == 0
+    need = lib.redmoe_workspace_bytes_host(C.byref(L), 1)
+
+    def fh(T=1, x=FAKE, out=FAKE, ids=FAKE, w=FAKE, ws=FAKE, ws_bytes=need):
+        return lib.redmoe_forward_host(C.byref(L), x, T, out, ids, w, ws, ws_bytes, 0)
+
+    assert fh(T=-1) == INVALID
+    assert fh(T=0) == OK
+    assert fh(x=None) == INVALID
+    assert fh(x=FAKE + 4) == INVALID
+    assert fh(out=FAKE + 8) == INVALID
+    assert fh(ids=FAKE + 2) == INVALID
+    assert fh(w=None) == INVALID
+    assert fh(ws=None) == WORKSPACE
+    assert fh(ws=FAKE + 128) == WORKSPACE
+    assert fh(ws_bytes=need - 256) == WORKSPACE
+    assert lib.redmoe_forward_host(C.byref(_layer(hidden=0)), FAKE, 1, FAKE, FAKE, FAKE, FAKE, need, 0) == INVALID
+
+
 def test_int4_layer_needs_scales(lib):
     L = _layer(expert_dtype=2)
     assert _fwd(lib, L) == INVALID
