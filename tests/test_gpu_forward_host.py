@@ -14,6 +14,8 @@ pytestmark = pytest.mark.gpu
 
 QWEN = mi.LayerShape(H=2048, E=512, k=10, I=512, Is=512)
 QWEN_INT4 = mi.LayerShape(H=2048, E=512, k=10, I=512, Is=512, expert_dtype="int4g32")
+QWEN_INT2 = mi.LayerShape(H=2048, E=512, k=10, I=512, Is=512, expert_dtype="int2g32")
+TINY = mi.WORKLOADS["tiny_f32"]["shape"]  # fp32 layer: the three- and four-row kernel at T = 1
 
 
 def _host_call(shape, L, x_dev, pinned=True):
@@ -46,6 +48,7 @@ def _device_call(shape, lay, x_dev):
 
 @pytest.mark.parametrize("shape,T,pinned", [
     (QWEN, 1, True), (QWEN, 1, False), (QWEN, 2, True), (QWEN, 3, True), (QWEN, 4, True), (QWEN_INT4, 1, True),
+    (QWEN_INT2, 1, True), (TINY, 1, True), (TINY, 3, True),
 ])
 def test_decode_sizes_match_device_buffers_and_oracle(gpu_lib, shape, T, pinned):
     L = mi.make_layer(shape, 7000 + T, "cuda")
