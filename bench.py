@@ -332,6 +332,16 @@ def cpu_oracle_prefill(wl, B, n=256):
                       f"({len(lay['w_gate'])} experts fetched), fp64, OpenMP over tokens"}
 
 
+def workload_config(wl, world):
+    """The `config` object both arms report for a workload."""
+    return {"workload": wl["desc"], "tokens_per_step": wl["T"], "layers": wl["layers"],
+            "layers_per_step": wl["layers"] if wl["stack"] else 1,
+            "l2": "inputs larger than L2: each step reads a different layer's weights "
+                  f"({wl['layers']} distinct layers)" if not wl["stack"] else
+                  f"inputs larger than L2: {wl['layers']} distinct layers per step",
+            "parallelism": "replicas" if world > 1 else "single GPU"}
+
+
 def reference_arm(args, wl, world, rank):
     """The fp64 oracle as the reference implementation, timed on the host cores."""
     import oracle
@@ -377,7 +387,8 @@ def reference_arm(args, wl, world, rank):
     return {"metric": METRIC, "value": value, "unit": unit, "n_gpus": 1, "steps": done, "warmup": args.warmup,
             "ms_per_step": 1e3 * el / max(done, 1), "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": wl["desc"], "tokens_per_step": tokens_per_step, "parallelism": "replicas"},
+            "config": {**workload_config(wl, world),
+                       "timing": "host wall clock around the timed steps (rank 0 alone runs this arm)"},
             "impl": "reference",
             "cpu_baseline": {"value": value, "unit": unit, "cores": cores, "kind": "oracle", "sample": sample},
             "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -536,12 +547,7 @@ def gpu_arm(args, wl, world, rank, local, B=None, name=None):
         "ms_per_step": el_ms / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": shape.expert_dtype,
         "data": "synthetic",
-        "config": {"workload": wl["desc"], "tokens_per_step": tokens_per_step, "layers": wl["layers"],
-                   "layers_per_step": wl["layers"] if wl["stack"] else 1,
-                   "l2": "inputs larger than L2: each step reads a different layer's weights "
-                         f"({wl['layers']} distinct layers)" if not wl["stack"] else
-                         f"inputs larger than L2: {wl['layers']} distinct layers per step",
-                   "parallelism": "replicas" if world > 1 else "single GPU",
+        "config": {**workload_config(wl, world),
                    "timing": "CUDA graph replay of exactly the timed steps (one graph up to 4096 steps); "
                              "untimed before it: the warm-up steps and one replay of the timed graph"},
         "roofline": roof,
