@@ -563,25 +563,21 @@ def e2e_arm(args, wl, smg, B, stream, world):
     nl = wl["layers"]
     K = args.steps
     xb = 4 if shape.x_dtype == "f32" else 2
-    xdt = torch.float32 if shape.x_dtype == "f32" else torch.bfloat16
     hx = [B["xs"][l].cpu().pin_memory() for l in range(nl)]
     hout = torch.empty(T, shape.H, dtype=torch.float32).pin_memory()
     hids = torch.empty(T, shape.k, dtype=torch.int32).pin_memory()
     hw = torch.empty(T, shape.k, dtype=torch.float32).pin_memory()
-    dx = [torch.empty(T, shape.H, dtype=xdt, device="cuda") for _ in range(nl)] if wl["stack"] else None
-    # one layer call per step: the host-buffer entry point (x staged by one copy; at decode
-    # sizes the kernel stores the results straight into the pinned host buffers)
-    wsh = None if wl["stack"] else smg.new_workspace_host(B["lays"][0], T)
+    # the host-buffer entry points: x comes in over the link (read by the kernel at T = 1,
+    # one copy otherwise) and the results land in the pinned host buffers
+    wsh = smg.new_workspace_host(B["lays"][0], T)
+    if wl["stack"]:
+        houts = [torch.empty(T, shape.H, dtype=torch.float32).pin_memory() for _ in range(nl)]
+        hidss = [torch.empty(T, shape.k, dtype=torch.int32).pin_memory() for _ in range(nl)]
+        hws = [torch.empty(T, shape.k, dtype=torch.float32).pin_memory() for _ in range(nl)]
 
     def step(i):
         if wl["stack"]:
-            for l in range(nl):
-                dx[l].copy_(hx[l], non_blocking=True)
-            smg.redmoe_forward_stack(B["lays"], dx, B["outs"], B["ids"], B["ws"], B["work"], stream=stream)
-            for l in range(nl):
-                hout.copy_(B["outs"][l], non_blocking=True)
-                hids.copy_(B["ids"][l], non_blocking=True)
-                hw.copy_(B["ws"][l], non_blocking=True)
+            smg.redmoe_forward_stack_host(B["lays"], hx, houts, hidss, hws, wsh, stream=stream)
         else:
             l = i % nl
             smg.redmoe_forward_host(B["lays"][l], hx[l], hout, hids, hw, wsh, stream=stream)
@@ -604,11 +600,10 @@ def e2e_arm(args, wl, smg, B, stream, world):
     d2h = (T * shape.H * 4 + T * shape.k * 8) * per
     return {"value": rate, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
             "d2h_bytes_per_step": d2h, "steps": n_e2e,
-            "how": ("redmoe_forward_stack through the C ABI per step; pinned host x copied in, out/ids/w copied "
-                    "out per layer" if wl["stack"] else
-                    "redmoe_forward_host through the C ABI per step: pinned host x copied in; out/ids/w land in "
-                    "pinned host buffers (stored by the kernel at T <= 4, copied back above)") +
-                   "; host wall clock around the K steps"}
+            "how": ("redmoe_forward_stack_host" if wl["stack"] else "redmoe_forward_host") +
+                   " through the C ABI per step, every x and result in pinned host memory: x read over the link "
+                   "by the kernel at T = 1 (copied in otherwise), results stored straight into the host buffers "
+                   "at T <= 4 (copied back otherwise); host wall clock around the K steps"}
 
 
 def host_link_gbs(nbytes=512 * 2**20, reps=5):

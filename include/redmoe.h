@@ -211,6 +211,19 @@ redmoe_status redmoe_forward_host(const redmoe_layer *L, const void *x_host, int
                                   int32_t *ids_host, float *w_host, void *workspace, size_t workspace_bytes,
                                   void *stream);
 
+/* redmoe_forward_stack with every x and every result in HOST memory (each array holds
+ * n_layers host pointers and lives in host memory). At T = 1 on the one-row kernel's
+ * layers, with every buffer pinned, the whole stack is one launch with no copy enqueued:
+ * the kernel reads each layer's x over the link at the layer's start and stores its
+ * results straight into the pinned buffers. Otherwise the layers run one after the other
+ * as redmoe_forward_host calls. Same rules and statuses as redmoe_forward_stack; the
+ * workspace must hold redmoe_workspace_bytes_host(&layers[0], T) bytes. The results are
+ * in host memory once `stream` has reached the end of the call. */
+redmoe_status redmoe_forward_stack_host(const redmoe_layer *layers, int32_t n_layers,
+                                        const void *const *xs, int32_t T, float *const *outs,
+                                        int32_t *const *ids, float *const *ws, void *workspace,
+                                        size_t workspace_bytes, void *stream);
+
 /* redmoe_forward for one token row (T = 1) whose routed expert stacks (w_gate, w_up,
  * w_down and their scales) may live in pinned host memory that the device can read
  * (cudaHostAlloc / cudaHostRegister, e.g. torch pin_memory); router, shared gate and

@@ -33,7 +33,7 @@ SYMBOLS = ("redmoe_abi_version", "redmoe_status_string", "redmoe_workspace_bytes
            "redmoe_check_timeout", "redmoe_forward_noalloc", "redmoe_selftest_wait_limit",
            "redmoe_fill_shared_memory", "redmoe_forward_cached", "redmoe_expert_cache_slot_bytes",
            "redmoe_expert_cache_init", "redmoe_forward_host_experts", "redmoe_expert_cache_prefetch",
-           "redmoe_workspace_bytes_host", "redmoe_forward_host")
+           "redmoe_workspace_bytes_host", "redmoe_forward_host", "redmoe_forward_stack_host")
 
 _lock = threading.Lock()
 _lib = None
@@ -117,6 +117,8 @@ def load():
         lib.redmoe_workspace_bytes_host.argtypes = [P, i32]
         lib.redmoe_forward_host.restype = i32
         lib.redmoe_forward_host.argtypes = [P, P, i32, P, P, P, P, sz, P]
+        lib.redmoe_forward_stack_host.restype = i32
+        lib.redmoe_forward_stack_host.argtypes = [P, i32, P, i32, P, P, P, P, sz, P]
         if lib.redmoe_abi_version() != ABI_VERSION:
             raise RuntimeError("libredmoe.so ABI version mismatch")
         _lib = lib
@@ -279,6 +281,23 @@ def redmoe_forward_stack(layers: Sequence[Layer], xs: Sequence[torch.Tensor], ou
                                      C.cast(P(*[_ptr(t) for t in ws]), C.c_void_p), _ptr(workspace),
                                      workspace.numel() * workspace.element_size(), _stream(stream))
     _check(st, "redmoe_forward_stack")
+
+
+def redmoe_forward_stack_host(layers: Sequence[Layer], xs: Sequence[torch.Tensor], outs: Sequence[torch.Tensor],
+                              ids: Sequence[torch.Tensor], ws: Sequence[torch.Tensor], workspace: torch.Tensor,
+                              stream=None) -> None:
+    """redmoe_forward_stack with every x and result in host memory (pinned for the
+    copy-free one-launch path); valid once `stream` has been synchronised."""
+    n = len(layers)
+    arr = (_Layer * n)(*[l.struct for l in layers])
+    P = C.c_void_p * n
+    T = xs[0].shape[0] if n else 0
+    st = load().redmoe_forward_stack_host(C.cast(arr, C.c_void_p), n, C.cast(P(*[_ptr(t) for t in xs]), C.c_void_p),
+                                          int(T), C.cast(P(*[_ptr(t) for t in outs]), C.c_void_p),
+                                          C.cast(P(*[_ptr(t) for t in ids]), C.c_void_p),
+                                          C.cast(P(*[_ptr(t) for t in ws]), C.c_void_p), _ptr(workspace),
+                                          workspace.numel() * workspace.element_size(), _stream(stream))
+    _check(st, "redmoe_forward_stack_host")
 
 
 def redmoe_check_timeout(workspace: Optional[torch.Tensor], stream=None) -> None:

@@ -264,7 +264,7 @@ redmoe_status redmoe_forward_host(const redmoe_layer* L, const void* x_host, int
         float* w = static_cast<float*>(writable_view(w_host));
         if (xv && o && i && w) {
             const DecLayer d = dec_layer(L, xv, o, i, w);
-            return launch_decode1_host_x(L, &d, workspace, base + h.x, s);
+            return launch_decode1_host_x(L, &d, 1, workspace, base + h.x, s);
         }
     }
     const size_t xbytes = (L->x_dtype == DT_F32 ? 4ull : 2ull) * T * L->hidden;
@@ -376,6 +376,53 @@ redmoe_status redmoe_forward_stack(const redmoe_layer* layers, int32_t n_layers,
     std::vector<DecLayer> d(n_layers);
     for (int l = 0; l < n_layers; ++l) d[l] = dec_layer(&layers[l], xs[l], outs[l], ids[l], ws[l]);
     return launch_decode(&layers[0], d.data(), n_layers, T, workspace, s, nullptr);
+}
+
+redmoe_status redmoe_forward_stack_host(const redmoe_layer* layers, int32_t n_layers, const void* const* xs,
+                                        int32_t T, float* const* outs, int32_t* const* ids, float* const* ws,
+                                        void* workspace, size_t workspace_bytes, void* stream) {
+    if (!layers || n_layers < 0 || !xs || !outs || !ids || !ws) return REDMOE_ERR_INVALID_ARG;
+    if (n_layers == 0 || T == 0) return T < 0 ? REDMOE_ERR_INVALID_ARG : REDMOE_OK;
+    if (T < 0) return REDMOE_ERR_INVALID_ARG;
+    redmoe_status st;
+    for (int l = 0; l < n_layers; ++l) {
+        if ((st = check_layer(&layers[l])) != REDMOE_OK) return st;
+        const redmoe_layer& a = layers[0];
+        const redmoe_layer& b = layers[l];
+        if (a.hidden != b.hidden || a.n_experts != b.n_experts || a.top_k != b.top_k || a.inter != b.inter ||
+            a.shared_inter != b.shared_inter || a.x_dtype != b.x_dtype || a.router_dtype != b.router_dtype ||
+            a.expert_dtype != b.expert_dtype)
+            return REDMOE_ERR_INVALID_ARG;
+        if (!xs[l] || !outs[l] || !ids[l] || !ws[l] || !aligned(xs[l], 16) || !aligned(outs[l], 16) ||
+            !aligned(ids[l], 4) || !aligned(ws[l], 4))
+            return REDMOE_ERR_INVALID_ARG;
+    }
+    if (!workspace || !aligned(workspace, 256)) return REDMOE_ERR_WORKSPACE;
+    const HostStage h = host_stage_layout(&layers[0], T);
+    if (workspace_bytes < h.total) return REDMOE_ERR_WORKSPACE;
+    if (T == 1 && decode1_shape_ok(&layers[0])) {
+        // one launch for the whole stack when every buffer is pinned: each layer's x is
+        // read over the link by the kernel and its results stored straight back
+        std::vector<DecLayer> d(n_layers);
+        bool mapped = true;
+        for (int l = 0; l < n_layers && mapped; ++l) {
+            const void* xv = writable_view(const_cast<void*>(xs[l]));
+            float* o = static_cast<float*>(writable_view(outs[l]));
+            int32_t* i = static_cast<int32_t*>(writable_view(ids[l]));
+            float* w = static_cast<float*>(writable_view(ws[l]));
+            mapped = xv && o && i && w;
+            if (mapped) d[l] = dec_layer(&layers[l], xv, o, i, w);
+        }
+        if (mapped)
+            return launch_decode1_host_x(&layers[0], d.data(), n_layers, workspace,
+                                         static_cast<char*>(workspace) + h.x, static_cast<cudaStream_t>(stream));
+    }
+    // otherwise layer by layer, each as redmoe_forward_host
+    for (int l = 0; l < n_layers; ++l)
+        if ((st = redmoe_forward_host(&layers[l], xs[l], T, outs[l], ids[l], ws[l], workspace, workspace_bytes,
+                                      stream)) != REDMOE_OK)
+            return st;
+    return REDMOE_OK;
 }
 
 redmoe_status redmoe_check_timeout(const void* workspace, void* stream) {

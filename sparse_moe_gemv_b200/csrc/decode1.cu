@@ -80,8 +80,10 @@ struct D1Params {
     float* hrt;     // [k, I]
     uint64_t timeout_ns;
     CacheBias cb;
-    // non-null: layer 0's x is pinned host memory (its device mapping in L[0].x); block 0
-    // copies it here and raises Control::x_ready, and every block reads it from here
+    // non-null: every layer's x is pinned host memory (its device mapping in L[l].x); at
+    // the start of each layer block 0 copies it here and counts on Control::x_ready, and
+    // every block reads it from here (one buffer: the barrier between stacked layers keeps
+    // a layer's copy from overwriting x that another block still reads)
     uint16_t* xstage;
     DecLayer L[NL];
 };
@@ -139,7 +141,7 @@ __global__ void __launch_bounds__(D1_THREADS, 1) decode1_kernel(const __grid_con
         const uint32_t par = uint32_t(l & 1);
 
         // ------------------------------------------------------------ phase A
-        const bool xremote = p.xstage != nullptr && l == 0;
+        const bool xremote = p.xstage != nullptr;
         if (xremote && blockIdx.x == 0 && warp >= 4) {
             // x from host memory: warps 4..7 of block 0 (no router row) read it once over the
             // link with cache-volatile loads (the host rewrites it between calls), every load
@@ -166,7 +168,7 @@ __global__ void __launch_bounds__(D1_THREADS, 1) decode1_kernel(const __grid_con
             const void* xsrc = x;
             if (xremote) {
                 const uint64_t t0 = globaltimer_ns();
-                for (uint32_t spins = 0; ld_acquire_gpu(&p.ctl->x_ready) < 4u; ++spins) {
+                for (uint32_t spins = 0; ld_acquire_gpu(&p.ctl->x_ready) < 4u * unsigned(l + 1); ++spins) {
                     if ((spins & 63u) == 63u && (globaltimer_ns() - t0 > to || spins > (1u << 26))) {
                         atomicOr(err, ERRBIT_TIMEOUT);
                         break;
@@ -491,7 +493,7 @@ redmoe_status d1_launch_all(const redmoe_layer* sh, const DecLayer* layers, int 
     }
     for (int l0 = 0; l0 < n_layers && st == REDMOE_OK; l0 += MAX_STACK) {
         const int n = n_layers - l0 < MAX_STACK ? n_layers - l0 : MAX_STACK;
-        st = d1_launch<WT, MAX_STACK>(sh, layers + l0, n, ws, stream, cb);
+        st = d1_launch<WT, MAX_STACK>(sh, layers + l0, n, ws, stream, cb, xstage);
         if (st == REDMOE_OK && launches) *launches += 1;
     }
     return st;
@@ -519,12 +521,12 @@ redmoe_status launch_decode1(const redmoe_layer* sh, const DecLayer* layers, int
     return d1_launch_all<DT_BF16>(sh, layers, n_layers, ws, stream, launches, cb);
 }
 
-redmoe_status launch_decode1_host_x(const redmoe_layer* sh, const DecLayer* layer, void* ws, void* xstage,
-                                    cudaStream_t stream) {
+redmoe_status launch_decode1_host_x(const redmoe_layer* sh, const DecLayer* layers, int n_layers, void* ws,
+                                    void* xstage, cudaStream_t stream) {
     const CacheBias cb{nullptr, 0.0f};
-    if (sh->expert_dtype == DT_INT4) return d1_launch_all<DT_INT4>(sh, layer, 1, ws, stream, nullptr, cb, xstage);
-    if (sh->expert_dtype == DT_INT2) return d1_launch_all<DT_INT2>(sh, layer, 1, ws, stream, nullptr, cb, xstage);
-    return d1_launch_all<DT_BF16>(sh, layer, 1, ws, stream, nullptr, cb, xstage);
+    if (sh->expert_dtype == DT_INT4) return d1_launch_all<DT_INT4>(sh, layers, n_layers, ws, stream, nullptr, cb, xstage);
+    if (sh->expert_dtype == DT_INT2) return d1_launch_all<DT_INT2>(sh, layers, n_layers, ws, stream, nullptr, cb, xstage);
+    return d1_launch_all<DT_BF16>(sh, layers, n_layers, ws, stream, nullptr, cb, xstage);
 }
 
 }  // namespace redmoe

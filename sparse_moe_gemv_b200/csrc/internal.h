@@ -72,10 +72,11 @@ DecodeWs decode_ws_layout(int T, int E, int k, int I, int Is);
 // The one-row kernel (T = 1, bf16 or int4 experts of the Qwen3-Next width): which layers
 // it takes, and its launch over n_layers layers.
 bool decode1_shape_ok(const redmoe_layer* sh);
-// One T = 1 layer whose x (layer->x) is the device mapping of pinned host memory: block 0
-// copies it into xstage (device, 2 H bytes, 16-byte aligned) and every block reads it there.
-redmoe_status launch_decode1_host_x(const redmoe_layer* sh, const DecLayer* layer, void* ws, void* xstage,
-                                    cudaStream_t stream);
+// T = 1 layers whose x (layers[l].x) is the device mapping of pinned host memory: block 0
+// copies each layer's x into xstage (device, 2 H bytes, 16-byte aligned) at the layer's
+// start and every block reads it there.
+redmoe_status launch_decode1_host_x(const redmoe_layer* sh, const DecLayer* layers, int n_layers, void* ws,
+                                    void* xstage, cudaStream_t stream);
 redmoe_status launch_decode1(const redmoe_layer* sh, const DecLayer* layers, int n_layers, void* ws,
                              cudaStream_t stream, int* launches, CacheBias cb);
 

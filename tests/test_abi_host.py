@@ -130,6 +130,24 @@ def test_forward_host_checks_before_touching_cuda(lib):
     assert lib.redmoe_forward_host(C.byref(_layer(hidden=0)), FAKE, 1, FAKE, FAKE, FAKE, FAKE, need, 0) == INVALID
 
 
+def test_forward_stack_host_checks_before_touching_cuda(lib):
+    L = _layer()
+    need = lib.redmoe_workspace_bytes_host(C.byref(L), 1)
+    arr = (smg._Layer * 2)(L, L)
+    P2 = C.c_void_p * 2
+
+    def fsh(n=2, T=1, x=FAKE, out=FAKE, ids=FAKE, w=FAKE, ws=FAKE, ws_bytes=need, layers=arr):
+        return lib.redmoe_forward_stack_host(C.cast(layers, C.c_void_p), n, C.cast(P2(x, x), C.c_void_p), T,
+                                             C.cast(P2(out, out), C.c_void_p), C.cast(P2(ids, ids), C.c_void_p),
+                                             C.cast(P2(w, w), C.c_void_p), ws, ws_bytes, 0)
+
+    assert fsh(n=0) == OK and fsh(T=0) == OK
+    assert fsh(n=-1) == INVALID and fsh(T=-1) == INVALID
+    assert fsh(x=FAKE + 4) == INVALID and fsh(out=FAKE + 8) == INVALID and fsh(ids=FAKE + 2) == INVALID
+    assert fsh(ws=None) == WORKSPACE and fsh(ws_bytes=need - 256) == WORKSPACE
+    assert fsh(layers=(smg._Layer * 2)(L, _layer(top_k=8))) == INVALID
+
+
 def test_int4_layer_needs_scales(lib):
     L = _layer(expert_dtype=2)
     assert _fwd(lib, L) == INVALID

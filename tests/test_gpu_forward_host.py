@@ -117,3 +117,39 @@ def test_rewritten_host_x_is_read_again(gpu_lib):
         dout, dids, dw = _device_call(shape, lay, x)
         assert torch.equal(hout, dout) and torch.equal(hids, dids) and torch.equal(hw, dw), seed
     smg.redmoe_check_timeout(ws)
+
+
+@pytest.mark.parametrize("shape,T,pinned", [
+    (QWEN, 1, True), (QWEN_INT4, 1, True), (QWEN_INT2, 1, True), (QWEN, 2, True), (QWEN, 1, False),
+])
+def test_stack_host_matches_device_stack(gpu_lib, shape, T, pinned):
+    """A stack of distinct layers with every x and result in host memory: one launch that
+    reads each layer's x over the link (T = 1, pinned), or layer-by-layer host calls;
+    either way bit for bit the device-buffer stack's results."""
+    n = 3
+    tens = [mi.make_layer(shape, 7500 + l, "cuda") for l in range(n)]
+    lays = [smg.Layer.from_shape(t, shape) for t in tens]
+    xs = [mi.make_x(shape, T, 7600 + l, "cuda") for l in range(n)]
+    dws = smg.new_workspace(lays[0], T)
+    douts = [torch.empty(T, shape.H, device="cuda") for _ in range(n)]
+    dids = [torch.empty(T, shape.k, dtype=torch.int32, device="cuda") for _ in range(n)]
+    dw = [torch.empty(T, shape.k, device="cuda") for _ in range(n)]
+    smg.redmoe_forward_stack(lays, xs, douts, dids, dw, dws)
+    torch.cuda.synchronize()
+
+    def host(t):
+        return t.pin_memory() if pinned else t
+    hxs = [host(x.cpu()) for x in xs]
+    houts = [host(torch.full((T, shape.H), float("nan"))) for _ in range(n)]
+    hids = [host(torch.full((T, shape.k), -1, dtype=torch.int32)) for _ in range(n)]
+    hw = [host(torch.full((T, shape.k), float("nan"))) for _ in range(n)]
+    ws = smg.new_workspace_host(lays[0], T)
+    s = torch.cuda.Stream()
+    smg.redmoe_forward_stack_host(lays, hxs, houts, hids, hw, ws, stream=s)
+    s.synchronize()
+    smg.redmoe_check_timeout(ws)
+    for l in range(n):
+        assert torch.equal(houts[l], douts[l].cpu()) and torch.equal(hids[l], dids[l].cpu()), l
+        assert torch.equal(hw[l], dw[l].cpu()), l
+    ot, wt = tolerances(shape)
+    assert_layer_parity(shape, tens[1], xs[1], houts[1].cuda(), hids[1].cuda(), hw[1].cuda(), ot, wt, "stack host layer 1")
