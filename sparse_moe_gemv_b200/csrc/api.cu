@@ -254,17 +254,18 @@ redmoe_status redmoe_forward_host(const redmoe_layer* L, const void* x_host, int
     if (workspace_bytes < h.total) return REDMOE_ERR_WORKSPACE;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     char* base = static_cast<char*>(workspace);
-    if (T == 1 && decode1_shape_ok(L)) {
-        // one token row with every buffer pinned: the kernel reads x over the link once
-        // (block 0 stages it in the workspace) and stores the results straight back, so no
-        // copy is enqueued at all
+    if ((T == 1 && decode1_shape_ok(L)) || decodefr_shape_ok(L, T)) {
+        // one or two token rows with every buffer pinned: the kernel reads x over the link
+        // once (staged in the workspace) and stores the results straight back, so no copy
+        // is enqueued at all
         const void* xv = writable_view(const_cast<void*>(x_host));
         float* o = static_cast<float*>(writable_view(out_host));
         int32_t* i = static_cast<int32_t*>(writable_view(ids_host));
         float* w = static_cast<float*>(writable_view(w_host));
         if (xv && o && i && w) {
             const DecLayer d = dec_layer(L, xv, o, i, w);
-            return launch_decode1_host_x(L, &d, 1, workspace, base + h.x, s);
+            return T == 1 ? launch_decode1_host_x(L, &d, 1, workspace, base + h.x, s)
+                          : launch_decodefr_host_x(L, &d, 1, T, workspace, base + h.x, s);
         }
     }
     const size_t xbytes = (L->x_dtype == DT_F32 ? 4ull : 2ull) * T * L->hidden;
@@ -400,7 +401,7 @@ redmoe_status redmoe_forward_stack_host(const redmoe_layer* layers, int32_t n_la
     if (!workspace || !aligned(workspace, 256)) return REDMOE_ERR_WORKSPACE;
     const HostStage h = host_stage_layout(&layers[0], T);
     if (workspace_bytes < h.total) return REDMOE_ERR_WORKSPACE;
-    if (T == 1 && decode1_shape_ok(&layers[0])) {
+    if ((T == 1 && decode1_shape_ok(&layers[0])) || decodefr_shape_ok(&layers[0], T)) {
         // one launch for the whole stack when every buffer is pinned: each layer's x is
         // read over the link by the kernel and its results stored straight back
         std::vector<DecLayer> d(n_layers);
@@ -413,9 +414,12 @@ redmoe_status redmoe_forward_stack_host(const redmoe_layer* layers, int32_t n_la
             mapped = xv && o && i && w;
             if (mapped) d[l] = dec_layer(&layers[l], xv, o, i, w);
         }
-        if (mapped)
-            return launch_decode1_host_x(&layers[0], d.data(), n_layers, workspace,
-                                         static_cast<char*>(workspace) + h.x, static_cast<cudaStream_t>(stream));
+        if (mapped) {
+            char* xstage = static_cast<char*>(workspace) + h.x;
+            cudaStream_t s = static_cast<cudaStream_t>(stream);
+            return T == 1 ? launch_decode1_host_x(&layers[0], d.data(), n_layers, workspace, xstage, s)
+                          : launch_decodefr_host_x(&layers[0], d.data(), n_layers, T, workspace, xstage, s);
+        }
     }
     // otherwise layer by layer, each as redmoe_forward_host
     for (int l = 0; l < n_layers; ++l)

@@ -80,6 +80,10 @@ struct FrParams {
     float* hrt;     // [T * k, I]   (row t * k + j: selection j of token t)
     uint64_t timeout_ns;
     CacheBias cb;
+    // non-null: every layer's x is pinned host memory (its device mapping in L[l].x); at
+    // each layer's start warp 7 of blocks 0 .. 2T-1 copies half a row each here and counts
+    // on Control::x_ready, and every x read of the layer comes from here
+    uint16_t* xstage;
     DecLayer L[NL];
 };
 
@@ -133,7 +137,8 @@ __global__ void __launch_bounds__(D1_THREADS, 1) decodefr_kernel(const __grid_co
 
     for (int l = 0; l < p.n_layers; ++l) {
         const DecLayer& Ly = p.L[l];
-        const uint16_t* x = static_cast<const uint16_t*>(Ly.x);
+        const bool xremote = p.xstage != nullptr;
+        const uint16_t* x = xremote ? p.xstage : static_cast<const uint16_t*>(Ly.x);
         float* sgate = p.sgate + (l & 1) * T;
         float* hsh = p.hsh + size_t(l & 1) * T * I;
         const uint32_t par = uint32_t(l & 1);
@@ -143,6 +148,41 @@ __global__ void __launch_bounds__(D1_THREADS, 1) decodefr_kernel(const __grid_co
             fence_proxy_async_smem();  // the previous layer's reads of the slots come first
             issue_down(0, Ly.sh_down, Ly.sh_s_down);
         }
+        bool xready = !xremote;  // this warp has seen the layer's x published
+        if (xremote && blockIdx.x < 2 * T && warp == D1_WARPS - 1) {
+            // x from host memory: half of row blockIdx.x / 2 per block, read once over the
+            // link with cache-volatile loads (the host rewrites it between calls), every load
+            // of a lane issued before its first store (one link round trip)
+            constexpr int PER = D1_XPL / 16;  // 16-byte chunks per lane: half a row per warp
+            const uint4* src = static_cast<const uint4*>(Ly.x) + size_t(blockIdx.x >> 1) * (H / 8);
+            uint4* dst = reinterpret_cast<uint4*>(p.xstage) + size_t(blockIdx.x >> 1) * (H / 8);
+            const int c0 = (blockIdx.x & 1) * (H / 16) + lane;
+            uint4 v[PER];
+#pragma unroll
+            for (int j = 0; j < PER; ++j)
+                if (32 * j + lane < H / 16) v[j] = __ldcv(src + c0 + 32 * j);
+#pragma unroll
+            for (int j = 0; j < PER; ++j)
+                if (32 * j + lane < H / 16) dst[c0 + 32 * j] = v[j];
+            __threadfence();
+            __syncwarp();
+            if (lane == 0) asm volatile("red.release.gpu.global.add.u32 [%0], 1;" :: "l"(&p.ctl->x_ready) : "memory");
+        }
+        // a warp's first x read of the layer waits until all 2T halves are published
+        auto wait_x = [&]() {
+            if (xready) return;
+            if (lane == 0) {
+                const uint64_t t0 = globaltimer_ns();
+                for (uint32_t spins = 0; ld_acquire_gpu(&p.ctl->x_ready) < 2u * T * unsigned(l + 1); ++spins) {
+                    if ((spins & 63u) == 63u && (globaltimer_ns() - t0 > to || spins > (1u << 26))) {
+                        atomicOr(err, ERRBIT_TIMEOUT);
+                        break;
+                    }
+                }
+            }
+            __syncwarp();
+            xready = true;
+        };
         for (int q = warp * nblocks + blockIdx.x; q < E + 1 + I; q += Wtot) {
             float2 a[T], b[T];
 #pragma unroll
@@ -153,7 +193,8 @@ __global__ void __launch_bounds__(D1_THREADS, 1) decodefr_kernel(const __grid_co
                 const void* row = q < E ? static_cast<const void*>(static_cast<const char*>(Ly.router_w) + size_t(q) * 2 * H)
                                         : Ly.shared_gate_w;
                 ld_row_bf(r, row, H, lane);
-                load_xp<DT_BF16, T>(x, H, lane, xp);
+                wait_x();
+                load_xp<DT_BF16, T, true>(x, H, lane, xp);
                 dotT_bf<T>(r, xp, (1u << T) - 1u, a);
 #pragma unroll
                 for (int t = 0; t < T; ++t) {
@@ -171,7 +212,8 @@ __global__ void __launch_bounds__(D1_THREADS, 1) decodefr_kernel(const __grid_co
                            PACKED ? Ly.sh_s_gate + size_t(i) * (H / 32) : nullptr, H, lane);
                 ld_row<WT>(u, static_cast<const char*>(Ly.sh_up) + size_t(i) * grow,
                            PACKED ? Ly.sh_s_up + size_t(i) * (H / 32) : nullptr, H, lane);
-                load_xp<WT, T>(x, H, lane, xp);
+                wait_x();
+                load_xp<WT, T, true>(x, H, lane, xp);
                 dotT<WT, T>(g, xp, (1u << T) - 1u, a);
                 dotT<WT, T>(u, xp, (1u << T) - 1u, b);
 #pragma unroll
@@ -322,7 +364,9 @@ __global__ void __launch_bounds__(D1_THREADS, 1) decodefr_kernel(const __grid_co
         }
         {
             uint32_t xp[T][32];
-            load_xp<WT, T>(x, H, lane, xp);
+            // (past the grid barrier: the layer's x is published whichever way it came;
+            // coherent loads throughout, since the staged x is written in this launch)
+            load_xp<WT, T, true>(x, H, lane, xp);
             constexpr int G = (WT == DT_BF16) ? 1 : (T == 2 ? 3 : 2);
             const int J = U * I;
             const int gw = blockIdx.x * D1_WARPS + warp;
@@ -461,7 +505,7 @@ int fr_blocks_per_sm(const void* kern, int smem) {
 
 template <int WT, int T, int NL>
 redmoe_status fr_launch(const redmoe_layer* sh, const DecLayer* layers, int n_layers, void* ws, cudaStream_t stream,
-                        CacheBias cb) {
+                        CacheBias cb, void* xstage) {
     DevInfo di;
     if (!get_dev_info(&di)) return REDMOE_ERR_CUDA;
     const int RB = (sh->hidden + di.sm_count - 1) / di.sm_count;
@@ -489,6 +533,7 @@ redmoe_status fr_launch(const redmoe_layer* sh, const DecLayer* layers, int n_la
     q.hrt = reinterpret_cast<float*>(base + L.hrt);
     q.timeout_ns = BARRIER_TIMEOUT_NS;
     q.cb = cb;
+    q.xstage = static_cast<uint16_t*>(xstage);
     for (int i = 0; i < n_layers; ++i) q.L[i] = layers[i];
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(di.sm_count * per_sm);
@@ -507,16 +552,16 @@ redmoe_status fr_launch(const redmoe_layer* sh, const DecLayer* layers, int n_la
 
 template <int WT, int T>
 redmoe_status fr_launch_all(const redmoe_layer* sh, const DecLayer* layers, int n_layers, void* ws, cudaStream_t stream,
-                            int* launches, CacheBias cb) {
+                            int* launches, CacheBias cb, void* xstage) {
     redmoe_status st = REDMOE_OK;
     if (n_layers == 1) {
-        st = fr_launch<WT, T, 1>(sh, layers, 1, ws, stream, cb);
+        st = fr_launch<WT, T, 1>(sh, layers, 1, ws, stream, cb, xstage);
         if (st == REDMOE_OK && launches) *launches += 1;
         return st;
     }
     for (int l0 = 0; l0 < n_layers && st == REDMOE_OK; l0 += MAX_STACK) {
         const int n = n_layers - l0 < MAX_STACK ? n_layers - l0 : MAX_STACK;
-        st = fr_launch<WT, T, MAX_STACK>(sh, layers + l0, n, ws, stream, cb);
+        st = fr_launch<WT, T, MAX_STACK>(sh, layers + l0, n, ws, stream, cb, xstage);
         if (st == REDMOE_OK && launches) *launches += 1;
     }
     return st;
@@ -524,10 +569,10 @@ redmoe_status fr_launch_all(const redmoe_layer* sh, const DecLayer* layers, int 
 
 template <int WT>
 redmoe_status fr_launch_t(const redmoe_layer* sh, const DecLayer* layers, int n_layers, int T, void* ws,
-                          cudaStream_t stream, int* launches, CacheBias cb) {
+                          cudaStream_t stream, int* launches, CacheBias cb, void* xstage = nullptr) {
     switch (T) {
-        case 2: return fr_launch_all<WT, 2>(sh, layers, n_layers, ws, stream, launches, cb);
-        case 3: return fr_launch_all<WT, 3>(sh, layers, n_layers, ws, stream, launches, cb);
+        case 2: return fr_launch_all<WT, 2>(sh, layers, n_layers, ws, stream, launches, cb, xstage);
+        case 3: return fr_launch_all<WT, 3>(sh, layers, n_layers, ws, stream, launches, cb, xstage);
         default: return REDMOE_ERR_UNSUPPORTED;
     }
 }
@@ -550,6 +595,13 @@ redmoe_status launch_decodefr(const redmoe_layer* sh, const DecLayer* layers, in
                               cudaStream_t stream, int* launches, CacheBias cb) {
     if (sh->expert_dtype == DT_INT4) return fr_launch_t<DT_INT4>(sh, layers, n_layers, T, ws, stream, launches, cb);
     return fr_launch_t<DT_BF16>(sh, layers, n_layers, T, ws, stream, launches, cb);
+}
+
+redmoe_status launch_decodefr_host_x(const redmoe_layer* sh, const DecLayer* layers, int n_layers, int T, void* ws,
+                                     void* xstage, cudaStream_t stream) {
+    const CacheBias cb{nullptr, 0.0f};
+    if (sh->expert_dtype == DT_INT4) return fr_launch_t<DT_INT4>(sh, layers, n_layers, T, ws, stream, nullptr, cb, xstage);
+    return fr_launch_t<DT_BF16>(sh, layers, n_layers, T, ws, stream, nullptr, cb, xstage);
 }
 
 }  // namespace redmoe

@@ -204,7 +204,8 @@ __host__ __device__ constexpr int d1_scale_bytes(int wt, int K) { return wt == D
 // elements 2m, 2m + 1 of the lane's slice (bf16: chunk c = lane + 32 j covers elements
 // 8c .. 8c + 7 -> words 4j .. 4j + 3; int4: chunk c covers 32c .. 32c + 31 -> words
 // 16j .. 16j + 15).
-template <int W, int T>
+// CG: coherent loads (x written earlier in the same launch), not the read-only path.
+template <int W, int T, bool CG = false>
 __device__ __forceinline__ void load_xp(const uint16_t* x, int H, int lane, uint32_t (&xp)[T][32]) {
     constexpr int PER = ChunkElems<W>::n;
     constexpr int NJ = D1_XPL / PER;
@@ -216,8 +217,8 @@ __device__ __forceinline__ void load_xp(const uint16_t* x, int H, int lane, uint
 #pragma unroll
             for (int q = 0; q < PER / 8; ++q) {
                 const int idx = c * PER + q * 8;
-                const uint4 v = idx < H ? __ldg(reinterpret_cast<const uint4*>(x + size_t(t) * H + idx))
-                                        : make_uint4(0u, 0u, 0u, 0u);
+                const uint4* px = reinterpret_cast<const uint4*>(x + size_t(t) * H + idx);
+                const uint4 v = idx < H ? (CG ? __ldcg(px) : __ldg(px)) : make_uint4(0u, 0u, 0u, 0u);
                 const int w = (j * (PER / 8) + q) * 4;
                 xp[t][w] = v.x;
                 xp[t][w + 1] = v.y;

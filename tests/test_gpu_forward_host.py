@@ -48,7 +48,7 @@ def _device_call(shape, lay, x_dev):
 
 @pytest.mark.parametrize("shape,T,pinned", [
     (QWEN, 1, True), (QWEN, 1, False), (QWEN, 2, True), (QWEN, 3, True), (QWEN, 4, True), (QWEN_INT4, 1, True),
-    (QWEN_INT2, 1, True), (TINY, 1, True), (TINY, 3, True),
+    (QWEN_INT2, 1, True), (TINY, 1, True), (TINY, 3, True), (QWEN_INT4, 2, True), (QWEN, 2, False),
 ])
 def test_decode_sizes_match_device_buffers_and_oracle(gpu_lib, shape, T, pinned):
     L = mi.make_layer(shape, 7000 + T, "cuda")
@@ -120,7 +120,8 @@ def test_rewritten_host_x_is_read_again(gpu_lib):
 
 
 @pytest.mark.parametrize("shape,T,pinned", [
-    (QWEN, 1, True), (QWEN_INT4, 1, True), (QWEN_INT2, 1, True), (QWEN, 2, True), (QWEN, 1, False),
+    (QWEN, 1, True), (QWEN_INT4, 1, True), (QWEN_INT2, 1, True), (QWEN, 2, True), (QWEN_INT4, 2, True),
+    (QWEN, 1, False), (QWEN, 3, True),
 ])
 def test_stack_host_matches_device_stack(gpu_lib, shape, T, pinned):
     """A stack of distinct layers with every x and result in host memory: one launch that
