@@ -81,13 +81,15 @@ struct FrParams {
     uint64_t timeout_ns;
     CacheBias cb;
     // non-null: every layer's x is pinned host memory (its device mapping in L[l].x); at
-    // each layer's start warp 7 of blocks 0 .. 2T-1 copies half a row each here and counts
+    // each layer's start warp 7 of blocks 0 .. 4T-1 copies a quarter row each here and counts
     // on Control::x_ready, and every x read of the layer comes from here
     uint16_t* xstage;
     DecLayer L[NL];
 };
 
-template <int WT, int T, int NL>
+// XR: x comes from pinned host memory through p.xstage (a separate instantiation, so
+// that calls on device buffers run without its waits and coherent loads).
+template <int WT, int T, int NL, bool XR>
 __global__ void __launch_bounds__(D1_THREADS, 1) decodefr_kernel(const __grid_constant__ FrParams<NL> p) {
     extern __shared__ __align__(128) unsigned char smem[];
     using Row = typename RowOf<WT>::type;
@@ -137,7 +139,7 @@ __global__ void __launch_bounds__(D1_THREADS, 1) decodefr_kernel(const __grid_co
 
     for (int l = 0; l < p.n_layers; ++l) {
         const DecLayer& Ly = p.L[l];
-        const bool xremote = p.xstage != nullptr;
+        constexpr bool xremote = XR;
         const uint16_t* x = xremote ? p.xstage : static_cast<const uint16_t*>(Ly.x);
         float* sgate = p.sgate + (l & 1) * T;
         float* hsh = p.hsh + size_t(l & 1) * T * I;
@@ -149,31 +151,31 @@ __global__ void __launch_bounds__(D1_THREADS, 1) decodefr_kernel(const __grid_co
             issue_down(0, Ly.sh_down, Ly.sh_s_down);
         }
         bool xready = !xremote;  // this warp has seen the layer's x published
-        if (xremote && blockIdx.x < 2 * T && warp == D1_WARPS - 1) {
-            // x from host memory: half of row blockIdx.x / 2 per block, read once over the
-            // link with cache-volatile loads (the host rewrites it between calls), every load
-            // of a lane issued before its first store (one link round trip)
-            constexpr int PER = D1_XPL / 16;  // 16-byte chunks per lane: half a row per warp
-            const uint4* src = static_cast<const uint4*>(Ly.x) + size_t(blockIdx.x >> 1) * (H / 8);
-            uint4* dst = reinterpret_cast<uint4*>(p.xstage) + size_t(blockIdx.x >> 1) * (H / 8);
-            const int c0 = (blockIdx.x & 1) * (H / 16) + lane;
+        if (xremote && blockIdx.x < 4 * T && warp == D1_WARPS - 1) {
+            // x from host memory: a quarter of row blockIdx.x / 4 per block, read once over
+            // the link with cache-volatile loads (the host rewrites it between calls), every
+            // load of a lane issued before its first store (one link round trip)
+            constexpr int PER = D1_XPL / 32;  // 16-byte chunks per lane: a quarter row per warp
+            const uint4* src = static_cast<const uint4*>(Ly.x) + size_t(blockIdx.x >> 2) * (H / 8);
+            uint4* dst = reinterpret_cast<uint4*>(p.xstage) + size_t(blockIdx.x >> 2) * (H / 8);
+            const int c0 = (blockIdx.x & 3) * (H / 32) + lane;
             uint4 v[PER];
 #pragma unroll
             for (int j = 0; j < PER; ++j)
-                if (32 * j + lane < H / 16) v[j] = __ldcv(src + c0 + 32 * j);
+                if (32 * j + lane < H / 32) v[j] = __ldcv(src + c0 + 32 * j);
 #pragma unroll
             for (int j = 0; j < PER; ++j)
-                if (32 * j + lane < H / 16) dst[c0 + 32 * j] = v[j];
+                if (32 * j + lane < H / 32) dst[c0 + 32 * j] = v[j];
             __threadfence();
             __syncwarp();
             if (lane == 0) asm volatile("red.release.gpu.global.add.u32 [%0], 1;" :: "l"(&p.ctl->x_ready) : "memory");
         }
-        // a warp's first x read of the layer waits until all 2T halves are published
+        // a warp's first x read of the layer waits until all 4T quarters are published
         auto wait_x = [&]() {
             if (xready) return;
             if (lane == 0) {
                 const uint64_t t0 = globaltimer_ns();
-                for (uint32_t spins = 0; ld_acquire_gpu(&p.ctl->x_ready) < 2u * T * unsigned(l + 1); ++spins) {
+                for (uint32_t spins = 0; ld_acquire_gpu(&p.ctl->x_ready) < 4u * T * unsigned(l + 1); ++spins) {
                     if ((spins & 63u) == 63u && (globaltimer_ns() - t0 > to || spins > (1u << 26))) {
                         atomicOr(err, ERRBIT_TIMEOUT);
                         break;
@@ -194,7 +196,7 @@ __global__ void __launch_bounds__(D1_THREADS, 1) decodefr_kernel(const __grid_co
                                         : Ly.shared_gate_w;
                 ld_row_bf(r, row, H, lane);
                 wait_x();
-                load_xp<DT_BF16, T, true>(x, H, lane, xp);
+                load_xp<DT_BF16, T, XR>(x, H, lane, xp);
                 dotT_bf<T>(r, xp, (1u << T) - 1u, a);
 #pragma unroll
                 for (int t = 0; t < T; ++t) {
@@ -213,7 +215,7 @@ __global__ void __launch_bounds__(D1_THREADS, 1) decodefr_kernel(const __grid_co
                 ld_row<WT>(u, static_cast<const char*>(Ly.sh_up) + size_t(i) * grow,
                            PACKED ? Ly.sh_s_up + size_t(i) * (H / 32) : nullptr, H, lane);
                 wait_x();
-                load_xp<WT, T, true>(x, H, lane, xp);
+                load_xp<WT, T, XR>(x, H, lane, xp);
                 dotT<WT, T>(g, xp, (1u << T) - 1u, a);
                 dotT<WT, T>(u, xp, (1u << T) - 1u, b);
 #pragma unroll
@@ -364,9 +366,9 @@ __global__ void __launch_bounds__(D1_THREADS, 1) decodefr_kernel(const __grid_co
         }
         {
             uint32_t xp[T][32];
-            // (past the grid barrier: the layer's x is published whichever way it came;
-            // coherent loads throughout, since the staged x is written in this launch)
-            load_xp<WT, T, true>(x, H, lane, xp);
+            // (past the grid barrier: the layer's x is published whichever way it came; the
+            // staged x is written in this launch, hence coherent loads)
+            load_xp<WT, T, XR>(x, H, lane, xp);
             constexpr int G = (WT == DT_BF16) ? 1 : (T == 2 ? 3 : 2);
             const int J = U * I;
             const int gw = blockIdx.x * D1_WARPS + warp;
@@ -503,7 +505,7 @@ int fr_blocks_per_sm(const void* kern, int smem) {
     return per_sm;
 }
 
-template <int WT, int T, int NL>
+template <int WT, int T, int NL, bool XR>
 redmoe_status fr_launch(const redmoe_layer* sh, const DecLayer* layers, int n_layers, void* ws, cudaStream_t stream,
                         CacheBias cb, void* xstage) {
     DevInfo di;
@@ -513,7 +515,7 @@ redmoe_status fr_launch(const redmoe_layer* sh, const DecLayer* layers, int n_la
     const int max_smem = di.max_smem_optin;
     const FrSmem S = fr_smem(WT, T, sh->top_k, sh->inter, RB, max_smem);
     if (S.nslot < 1 || S.total > max_smem) return REDMOE_ERR_UNSUPPORTED;
-    auto kern = decodefr_kernel<WT, T, NL>;
+    auto kern = decodefr_kernel<WT, T, NL, XR>;
     const int per_sm = fr_blocks_per_sm(reinterpret_cast<const void*>(kern), S.total);
     if (per_sm < 0) return REDMOE_ERR_CUDA;
     if (per_sm == 0) return REDMOE_ERR_UNSUPPORTED;
@@ -550,18 +552,18 @@ redmoe_status fr_launch(const redmoe_layer* sh, const DecLayer* layers, int n_la
     return err == cudaSuccess ? REDMOE_OK : REDMOE_ERR_CUDA;
 }
 
-template <int WT, int T>
+template <int WT, int T, bool XR>
 redmoe_status fr_launch_all(const redmoe_layer* sh, const DecLayer* layers, int n_layers, void* ws, cudaStream_t stream,
                             int* launches, CacheBias cb, void* xstage) {
     redmoe_status st = REDMOE_OK;
     if (n_layers == 1) {
-        st = fr_launch<WT, T, 1>(sh, layers, 1, ws, stream, cb, xstage);
+        st = fr_launch<WT, T, 1, XR>(sh, layers, 1, ws, stream, cb, xstage);
         if (st == REDMOE_OK && launches) *launches += 1;
         return st;
     }
     for (int l0 = 0; l0 < n_layers && st == REDMOE_OK; l0 += MAX_STACK) {
         const int n = n_layers - l0 < MAX_STACK ? n_layers - l0 : MAX_STACK;
-        st = fr_launch<WT, T, MAX_STACK>(sh, layers + l0, n, ws, stream, cb, xstage);
+        st = fr_launch<WT, T, MAX_STACK, XR>(sh, layers + l0, n, ws, stream, cb, xstage);
         if (st == REDMOE_OK && launches) *launches += 1;
     }
     return st;
@@ -569,10 +571,10 @@ redmoe_status fr_launch_all(const redmoe_layer* sh, const DecLayer* layers, int 
 
 template <int WT>
 redmoe_status fr_launch_t(const redmoe_layer* sh, const DecLayer* layers, int n_layers, int T, void* ws,
-                          cudaStream_t stream, int* launches, CacheBias cb, void* xstage = nullptr) {
+                          cudaStream_t stream, int* launches, CacheBias cb) {
     switch (T) {
-        case 2: return fr_launch_all<WT, 2>(sh, layers, n_layers, ws, stream, launches, cb, xstage);
-        case 3: return fr_launch_all<WT, 3>(sh, layers, n_layers, ws, stream, launches, cb, xstage);
+        case 2: return fr_launch_all<WT, 2, false>(sh, layers, n_layers, ws, stream, launches, cb, nullptr);
+        case 3: return fr_launch_all<WT, 3, false>(sh, layers, n_layers, ws, stream, launches, cb, nullptr);
         default: return REDMOE_ERR_UNSUPPORTED;
     }
 }
@@ -600,8 +602,10 @@ redmoe_status launch_decodefr(const redmoe_layer* sh, const DecLayer* layers, in
 redmoe_status launch_decodefr_host_x(const redmoe_layer* sh, const DecLayer* layers, int n_layers, int T, void* ws,
                                      void* xstage, cudaStream_t stream) {
     const CacheBias cb{nullptr, 0.0f};
-    if (sh->expert_dtype == DT_INT4) return fr_launch_t<DT_INT4>(sh, layers, n_layers, T, ws, stream, nullptr, cb, xstage);
-    return fr_launch_t<DT_BF16>(sh, layers, n_layers, T, ws, stream, nullptr, cb, xstage);
+    if (T != 2) return REDMOE_ERR_UNSUPPORTED;  // the host-memory x instantiations are built for T = 2
+    if (sh->expert_dtype == DT_INT4)
+        return fr_launch_all<DT_INT4, 2, true>(sh, layers, n_layers, ws, stream, nullptr, cb, xstage);
+    return fr_launch_all<DT_BF16, 2, true>(sh, layers, n_layers, ws, stream, nullptr, cb, xstage);
 }
 
 }  // namespace redmoe

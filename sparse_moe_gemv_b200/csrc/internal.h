@@ -85,7 +85,7 @@ bool decodefr_shape_ok(const redmoe_layer* sh, int T);
 redmoe_status launch_decodefr(const redmoe_layer* sh, const DecLayer* layers, int n_layers, int T, void* ws,
                               cudaStream_t stream, int* launches, CacheBias cb);
 // The same with every layer's x (layers[l].x, T rows) the device mapping of pinned host
-// memory: blocks 0 .. 2T-1 copy it into xstage (device, T * 2 H bytes, 16-byte aligned)
+// memory: blocks 0 .. 4T-1 copy it into xstage (device, T * 2 H bytes, 16-byte aligned)
 // at each layer's start and every x read comes from there.
 redmoe_status launch_decodefr_host_x(const redmoe_layer* sh, const DecLayer* layers, int n_layers, int T, void* ws,
                                      void* xstage, cudaStream_t stream);
