@@ -88,7 +88,9 @@ struct D1Params {
     DecLayer L[NL];
 };
 
-template <int WT, int NL>
+// XR: every layer's x comes from pinned host memory through p.xstage (a separate
+// instantiation, so that calls on device buffers carry none of that code).
+template <int WT, int NL, bool XR>
 __global__ void __launch_bounds__(D1_THREADS, 1) decode1_kernel(const __grid_constant__ D1Params<NL> p) {
     extern __shared__ __align__(128) unsigned char smem[];
     using Row = typename RowOf<WT>::type;
@@ -141,7 +143,7 @@ __global__ void __launch_bounds__(D1_THREADS, 1) decode1_kernel(const __grid_con
         const uint32_t par = uint32_t(l & 1);
 
         // ------------------------------------------------------------ phase A
-        const bool xremote = p.xstage != nullptr;
+        constexpr bool xremote = XR;
         if (xremote && blockIdx.x == 0 && warp >= 4) {
             // x from host memory: warps 4..7 of block 0 (no router row) read it once over the
             // link with cache-volatile loads (the host rewrites it between calls), every load
@@ -435,16 +437,16 @@ int d1_blocks_per_sm(const void* kern, int smem) {
     return per_sm;
 }
 
-template <int WT, int NL>
+template <int WT, int NL, bool XR>
 redmoe_status d1_launch(const redmoe_layer* sh, const DecLayer* layers, int n_layers, void* ws, cudaStream_t stream,
-                        CacheBias cb, void* xstage = nullptr) {
+                        CacheBias cb, void* xstage) {
     DevInfo di;
     if (!get_dev_info(&di)) return REDMOE_ERR_CUDA;
     const int RB = (sh->hidden + di.sm_count - 1) / di.sm_count;
     if (RB > D1_RB_MAX) return REDMOE_ERR_UNSUPPORTED;
     const D1Smem S = d1_smem(WT, sh->top_k, sh->inter, RB, sh->hidden);
     if (S.total > di.max_smem_optin) return REDMOE_ERR_UNSUPPORTED;
-    auto kern = decode1_kernel<WT, NL>;
+    auto kern = decode1_kernel<WT, NL, XR>;
     const int per_sm = d1_blocks_per_sm(reinterpret_cast<const void*>(kern), S.total);
     if (per_sm < 0) return REDMOE_ERR_CUDA;
     if (per_sm == 0) return REDMOE_ERR_UNSUPPORTED;
@@ -482,18 +484,18 @@ redmoe_status d1_launch(const redmoe_layer* sh, const DecLayer* layers, int n_la
     return err == cudaSuccess ? REDMOE_OK : REDMOE_ERR_CUDA;
 }
 
-template <int WT>
+template <int WT, bool XR = false>
 redmoe_status d1_launch_all(const redmoe_layer* sh, const DecLayer* layers, int n_layers, void* ws, cudaStream_t stream,
                             int* launches, CacheBias cb, void* xstage = nullptr) {
     redmoe_status st = REDMOE_OK;
     if (n_layers == 1) {
-        st = d1_launch<WT, 1>(sh, layers, 1, ws, stream, cb, xstage);
+        st = d1_launch<WT, 1, XR>(sh, layers, 1, ws, stream, cb, xstage);
         if (st == REDMOE_OK && launches) *launches += 1;
         return st;
     }
     for (int l0 = 0; l0 < n_layers && st == REDMOE_OK; l0 += MAX_STACK) {
         const int n = n_layers - l0 < MAX_STACK ? n_layers - l0 : MAX_STACK;
-        st = d1_launch<WT, MAX_STACK>(sh, layers + l0, n, ws, stream, cb, xstage);
+        st = d1_launch<WT, MAX_STACK, XR>(sh, layers + l0, n, ws, stream, cb, xstage);
         if (st == REDMOE_OK && launches) *launches += 1;
     }
     return st;
@@ -524,9 +526,9 @@ redmoe_status launch_decode1(const redmoe_layer* sh, const DecLayer* layers, int
 redmoe_status launch_decode1_host_x(const redmoe_layer* sh, const DecLayer* layers, int n_layers, void* ws,
                                     void* xstage, cudaStream_t stream) {
     const CacheBias cb{nullptr, 0.0f};
-    if (sh->expert_dtype == DT_INT4) return d1_launch_all<DT_INT4>(sh, layers, n_layers, ws, stream, nullptr, cb, xstage);
-    if (sh->expert_dtype == DT_INT2) return d1_launch_all<DT_INT2>(sh, layers, n_layers, ws, stream, nullptr, cb, xstage);
-    return d1_launch_all<DT_BF16>(sh, layers, n_layers, ws, stream, nullptr, cb, xstage);
+    if (sh->expert_dtype == DT_INT4) return d1_launch_all<DT_INT4, true>(sh, layers, n_layers, ws, stream, nullptr, cb, xstage);
+    if (sh->expert_dtype == DT_INT2) return d1_launch_all<DT_INT2, true>(sh, layers, n_layers, ws, stream, nullptr, cb, xstage);
+    return d1_launch_all<DT_BF16, true>(sh, layers, n_layers, ws, stream, nullptr, cb, xstage);
 }
 
 }  // namespace redmoe
