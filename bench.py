@@ -57,7 +57,7 @@ WORKLOADS = {
                       desc="Qwen3-Next-shaped MoE layer, bf16 weights / fp32 accumulate, decode T=1"),
     "fewrow_t2": dict(shape=QWEN, T=2, layers=12, stack=True, seed=2000, kernel="decodefr_kernel",
                       desc="12 distinct Qwen3-Next-shaped bf16 layers back to back, T=2"),
-    "fewrow_t3": dict(shape=QWEN, T=3, layers=12, stack=True, seed=2000, kernel="decode_kernel",
+    "fewrow_t3": dict(shape=QWEN, T=3, layers=12, stack=True, seed=2000, kernel="decodefr_kernel + decode1_kernel",
                       desc="12 distinct Qwen3-Next-shaped bf16 layers back to back, T=3"),
     "int4_48": dict(shape=QWEN_INT4, T=1, layers=48, stack=True, seed=4000, kernel="decode1_kernel",
                     desc="48 distinct Qwen3-Next-shaped layers, int4 group-32 experts, decode T=1"),
@@ -412,15 +412,18 @@ def build_workload(wl, smg, tens=None):
 def make_step(wl, smg, B, stream):
     """step(i): the i-th step's launches on `stream`."""
     nl = wl["layers"]
+    shape = wl["shape"]
+    # three and four rows run as rows 0-1 on the few-row kernel plus the rest: two launches
+    split = 2 if wl["T"] in (3, 4) and shape.x_dtype == "bf16" and shape.expert_dtype in ("bf16", "int4g32") else 1
     if wl["stack"]:
         def step(i):
             smg.redmoe_forward_stack(B["lays"], B["xs"], B["outs"], B["ids"], B["ws"], B["work"], stream=stream)
-        return step, 1 if nl <= 64 else math.ceil(nl / 64)
+        return step, split * (1 if nl <= 64 else math.ceil(nl / 64))
 
     def step(i):
         l = i % nl
         smg.redmoe_forward(B["lays"][l], B["xs"][l], B["outs"][l], B["ids"][l], B["ws"][l], B["work"], stream=stream)
-    return step, 1
+    return step, split
 
 
 def capture(step, n, stream):
@@ -504,14 +507,16 @@ def gpu_arm(args, wl, world, rank, local, B=None, name=None):
     el_ms = max_over_ranks(el_ms, world)
 
     distinct = distinct_experts(B)
+    # algorithmic bytes of one step: the whole stack, or one layer call (averaged over the
+    # rotation's layers)
     if wl["stack"]:
-        bytes_per_launch = sum(layer_call_bytes(shape, T, d) for d in distinct)
+        bytes_per_step = sum(layer_call_bytes(shape, T, d) for d in distinct)
     else:
-        bytes_per_launch = sum(layer_call_bytes(shape, T, d) for d in distinct) / len(distinct)
+        bytes_per_step = sum(layer_call_bytes(shape, T, d) for d in distinct) / len(distinct)
     launches = K * launches_per_step
-    launch_s = el_ms / 1e3 / launches
+    step_s = el_ms / 1e3 / K
     hbm, bf16, bf16_sus, src = peaks()
-    achieved = bytes_per_launch / launch_s / 1e9
+    achieved = bytes_per_step / step_s / 1e9
     key = name or args.workload
     if T > 4:
         # batched path: four kernels per step. Its roofline is the binding one of two: the
@@ -519,12 +524,11 @@ def gpu_arm(args, wl, world, rank, local, B=None, name=None):
         # peak, and its FLOPs at the bf16 tensor peak. With a few tokens per expert the
         # weights dominate and the HBM time is the larger.
         flops = layer_flops(shape, T)
-        step_s = el_ms / 1e3 / K
         tfl = flops / step_s / 1e12
-        gbs = bytes_per_launch / step_s / 1e9
-        t_hbm, t_tc = bytes_per_launch / (hbm * 1e9), flops / (bf16 * 1e12)
+        gbs = bytes_per_step / step_s / 1e9
+        t_hbm, t_tc = bytes_per_step / (hbm * 1e9), flops / (bf16 * 1e12)
         both = {"traffic": profile_traffic(key), "kernel": wl["kernel"], "flops_per_step": flops,
-                "bytes_per_step": bytes_per_launch, "hbm_floor_us": t_hbm * 1e6, "tensor_floor_us": t_tc * 1e6,
+                "bytes_per_step": bytes_per_step, "hbm_floor_us": t_hbm * 1e6, "tensor_floor_us": t_tc * 1e6,
                 "tensor_tflops": tfl, "tensor_frac": tfl / bf16, "hbm_gbs": gbs, "hbm_frac": gbs / hbm}
         if t_hbm >= t_tc:
             roof = {"bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s", "frac": gbs / hbm, **both,
@@ -536,8 +540,8 @@ def gpu_arm(args, wl, world, rank, local, B=None, name=None):
     else:
         roof = {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
                 "traffic": profile_traffic(key, wl["layers"] if wl["stack"] else 1), "kernel": wl["kernel"],
-                "bytes_per_launch": bytes_per_launch,
-                "launch_us": launch_s * 1e6, "distinct_experts_per_layer": statistics.mean(distinct),
+                "bytes_per_step": bytes_per_step, "step_us": step_s * 1e6,
+                "launches_per_step": launches_per_step, "distinct_experts_per_layer": statistics.mean(distinct),
                 "peak_source": f"{src} (MEASURED_PEAKS.json hbm_gbs)" if src == "measured" else "fallback"}
 
     # end to end through the C ABI with pinned host buffers: per step H2D x, forward, D2H out/ids/w

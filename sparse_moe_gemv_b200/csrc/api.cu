@@ -242,6 +242,24 @@ void* writable_view(void* p) {
     return nullptr;
 }
 
+// The decode launches of host-memory x (layers[l].x mapped pinned memory, T rows staged at
+// xstage): T = 1 and 2 on their kernels, T = 3 and 4 as rows 0-1 plus the rest.
+redmoe_status launch_decode_host_x(const redmoe_layer* L, const DecLayer* d, int n, int T, void* ws, char* xstage,
+                                   cudaStream_t s) {
+    if (T == 1) return launch_decode1_host_x(L, d, n, ws, xstage, s);
+    if (T == 2) return launch_decodefr_host_x(L, d, n, 2, ws, xstage, s);
+    redmoe_status st = launch_decodefr_host_x(L, d, n, 2, ws, xstage, s);
+    if (st != REDMOE_OK) return st;
+    const std::vector<DecLayer> rest = dec_rows(L, d, n, 2);
+    char* xs2 = xstage + size_t(2) * L->hidden * (L->x_dtype == DT_F32 ? 4 : 2);
+    return T == 3 ? launch_decode1_host_x(L, rest.data(), n, ws, xs2, s)
+                  : launch_decodefr_host_x(L, rest.data(), n, 2, ws, xs2, s);
+}
+
+bool host_x_ok(const redmoe_layer* L, int T) {
+    return (T == 1 && decode1_shape_ok(L)) || decodefr_shape_ok(L, T) || decode_split_ok(L, T);
+}
+
 }  // namespace
 
 size_t redmoe_workspace_bytes_host(const redmoe_layer* L, int32_t T) {
@@ -264,18 +282,17 @@ redmoe_status redmoe_forward_host(const redmoe_layer* L, const void* x_host, int
     if (workspace_bytes < h.total) return REDMOE_ERR_WORKSPACE;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     char* base = static_cast<char*>(workspace);
-    if ((T == 1 && decode1_shape_ok(L)) || decodefr_shape_ok(L, T)) {
-        // one or two token rows with every buffer pinned: the kernel reads x over the link
-        // once (staged in the workspace) and stores the results straight back, so no copy
-        // is enqueued at all
+    if (host_x_ok(L, T)) {
+        // decode rows with every buffer pinned: the kernels read x over the link once
+        // (staged in the workspace) and store the results straight back, so no copy is
+        // enqueued at all
         const void* xv = writable_view(const_cast<void*>(x_host));
         float* o = static_cast<float*>(writable_view(out_host));
         int32_t* i = static_cast<int32_t*>(writable_view(ids_host));
         float* w = static_cast<float*>(writable_view(w_host));
         if (xv && o && i && w) {
             const DecLayer d = dec_layer(L, xv, o, i, w);
-            return T == 1 ? launch_decode1_host_x(L, &d, 1, workspace, base + h.x, s)
-                          : launch_decodefr_host_x(L, &d, 1, T, workspace, base + h.x, s);
+            return launch_decode_host_x(L, &d, 1, T, workspace, base + h.x, s);
         }
     }
     const size_t xbytes = (L->x_dtype == DT_F32 ? 4ull : 2ull) * T * L->hidden;
@@ -419,7 +436,7 @@ redmoe_status redmoe_forward_stack_host(const redmoe_layer* layers, int32_t n_la
     if (!workspace || !aligned(workspace, 256)) return REDMOE_ERR_WORKSPACE;
     const HostStage h = host_stage_layout(&layers[0], T);
     if (workspace_bytes < h.total) return REDMOE_ERR_WORKSPACE;
-    if ((T == 1 && decode1_shape_ok(&layers[0])) || decodefr_shape_ok(&layers[0], T)) {
+    if (host_x_ok(&layers[0], T)) {
         // one launch for the whole stack when every buffer is pinned: each layer's x is
         // read over the link by the kernel and its results stored straight back
         std::vector<DecLayer> d(n_layers);
@@ -432,12 +449,9 @@ redmoe_status redmoe_forward_stack_host(const redmoe_layer* layers, int32_t n_la
             mapped = xv && o && i && w;
             if (mapped) d[l] = dec_layer(&layers[l], xv, o, i, w);
         }
-        if (mapped) {
-            char* xstage = static_cast<char*>(workspace) + h.x;
-            cudaStream_t s = static_cast<cudaStream_t>(stream);
-            return T == 1 ? launch_decode1_host_x(&layers[0], d.data(), n_layers, workspace, xstage, s)
-                          : launch_decodefr_host_x(&layers[0], d.data(), n_layers, T, workspace, xstage, s);
-        }
+        if (mapped)
+            return launch_decode_host_x(&layers[0], d.data(), n_layers, T, workspace,
+                                        static_cast<char*>(workspace) + h.x, static_cast<cudaStream_t>(stream));
     }
     // otherwise layer by layer, each as redmoe_forward_host
     for (int l = 0; l < n_layers; ++l)

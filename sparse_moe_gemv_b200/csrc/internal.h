@@ -1,6 +1,8 @@
 // Declarations shared between the .cu files of libredmoe (not part of the C ABI).
 #pragma once
 
+#include <vector>
+
 #include <cuda_runtime.h>
 #include <stddef.h>
 #include <stdint.h>
@@ -55,6 +57,11 @@ struct DecLayer {
 
 // The decode kernel's view of one redmoe_layer called on (x, out, ids, w).
 DecLayer dec_layer(const redmoe_layer* L, const void* x, float* out, int32_t* ids, float* w);
+// The same calls restricted to rows r0 .. of x, out, ids and w.
+std::vector<DecLayer> dec_rows(const redmoe_layer* sh, const DecLayer* layers, int n_layers, int r0);
+// Decode sizes run as rows 0-1 on the few-row kernel plus the rest on the one- or few-row
+// kernel (T = 3, 4 on layers both take).
+bool decode_split_ok(const redmoe_layer* sh, int T);
 
 // Layer validation shared by every entry point (shape, dtype combination, pointers).
 redmoe_status check_layer(const redmoe_layer* L);
