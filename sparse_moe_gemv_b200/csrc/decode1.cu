@@ -48,6 +48,25 @@ namespace {
 
 __device__ __forceinline__ float hsum2(float2 v) { return warp_sum(v.x + v.y); }
 
+// Word of h element i (I = 512) in a staged h row. In phase C lane l holds the 16
+// elements its chunk of a down row covers: l*16 .. l*16+15 for int4 and int2 rows (one 8-
+// or 4-byte load), and l*8 .. l*8+7 with 256+l*8 .. 256+l*8+7 for bf16 rows (two 16-byte
+// loads 512 bytes apart, each conflict-free over the warp). Element m of lane l sits at
+// word 128*(m/4) + 4*l + m%4, so that the lane's four 16-byte loads of h are
+// conflict-free too.
+template <int WT>
+__device__ __forceinline__ int hpos(int i) {
+    int l, m;
+    if constexpr (WT == DT_BF16) {
+        l = (i & 255) >> 3;
+        m = (i & 7) | ((i >> 8) << 3);
+    } else {
+        l = i >> 4;
+        m = i & 15;
+    }
+    return 128 * (m >> 2) + 4 * l + (m & 3);
+}
+
 // Shared-memory plan of the kernel (byte offsets). `dreg` holds the block's rows of the
 // down matrix of k + 1 experts (routed slots 0..k-1 in selection order, the shared
 // expert in slot k), each slot RB rows (int4: codes, then scales).
@@ -65,7 +84,7 @@ __host__ __device__ inline D1Smem d1_smem(int wt, int k, int I, int RB, int H) {
     s.xs = o; o += a16(2 * H);  // the layer's x (bf16), one bulk copy per layer
     s.bars = o; o += 8 * (D1_MAXK + 3);
     s.part = o; o += 4 * D1_WARPS * D1_RB_MAX;
-    s.sel = o; o += 12 * D1_MAXK;  // the block's top-k: ids, weights, stack indices
+    s.sel = o; o += 12 * D1_MAXK + 4;  // the block's top-k: ids, weights, stack indices; the shared gate
     s.total = a16(o);
     return s;
 }
@@ -110,6 +129,7 @@ __global__ void __launch_bounds__(D1_THREADS, 1) decode1_kernel(const __grid_con
     int* s_sel_id = reinterpret_cast<int*>(smem + S.sel);
     float* s_sel_w = reinterpret_cast<float*>(smem + S.sel) + D1_MAXK;
     int* s_sel_slot = reinterpret_cast<int*>(smem + S.sel) + 2 * D1_MAXK;
+    float* s_wsh = reinterpret_cast<float*>(smem + S.sel) + 3 * D1_MAXK;
     constexpr bool PACKED = WT != DT_BF16;           // int4 / int2: codes plus group scales
     const int drow = d1_row_bytes(WT, I);            // bytes of one down row (codes)
     const int dsc = d1_scale_bytes(WT, I);           // bytes of its scales
@@ -223,7 +243,7 @@ __global__ void __launch_bounds__(D1_THREADS, 1) decode1_kernel(const __grid_con
             mbar_wait(xbar, par, err, to);
             load_x<WT, true>(reinterpret_cast<const uint16_t*>(smem + S.xs), H, lane, xr);
             const float a = hsum2(dot_row<WT>(g, xr)), b = hsum2(dot_row<WT>(u, xr));
-            if (lane == 0) hsh[i] = silu_mul(a, b);
+            if (lane == 0) hsh[hpos<WT>(i)] = silu_mul(a, b);
         }
 
         // Phase C's work comes in units (slot u, half hf of the block's rows): 2 (k + 1)
@@ -253,8 +273,9 @@ __global__ void __launch_bounds__(D1_THREADS, 1) decode1_kernel(const __grid_con
                         const float2 b = dot8_q4(wv.y, hf32 + 8, make_float2(0.f, 0.f));
                         d = ffma2(make_float2(s, s), fadd2(a, b), d);
                     } else {
-                        const uint4* wr = reinterpret_cast<const uint4*>(slot + (ra + r) * drow + lane * 32);
-                        const uint4 w0 = wr[0], w1 = wr[1];
+                        const unsigned char* wr = slot + (ra + r) * drow + lane * 16;
+                        const uint4 w0 = *reinterpret_cast<const uint4*>(wr);
+                        const uint4 w1 = *reinterpret_cast<const uint4*>(wr + 512);
                         float2 e = make_float2(0.f, 0.f);
                         d = ffma2(bf2(w0.x), make_float2(hf32[0], hf32[1]), d);
                         e = ffma2(bf2(w0.y), make_float2(hf32[2], hf32[3]), e);
@@ -275,6 +296,7 @@ __global__ void __launch_bounds__(D1_THREADS, 1) decode1_kernel(const __grid_con
             // one warp per block takes the top-k of the logits (lane j < k: id and
             // renormalised weight of selection j) and shares it
             grid_wait_warp(p.ctl, nblocks, bar1, to);
+            const float sg = __ldcg(sgate);  // the shared expert's gate, read beside the logits
             int id = 0;
             float wv = 0.0f;
             if (Ly.given_ids) {
@@ -297,6 +319,7 @@ __global__ void __launch_bounds__(D1_THREADS, 1) decode1_kernel(const __grid_con
                 s_sel_id[lane] = id;
                 s_sel_w[lane] = wv;
                 s_sel_slot[lane] = slot;
+                if (lane == 0) *s_wsh = sg;
                 if (blockIdx.x == 0) {
                     Ly.ids[lane] = id;
                     Ly.w[lane] = wv;
@@ -349,7 +372,7 @@ __global__ void __launch_bounds__(D1_THREADS, 1) decode1_kernel(const __grid_con
                     const int j = jb + t * Wtot;
                     if (j < J) {
                         const float a = hsum2(dot_row<WT>(g[t], xf)), b = hsum2(dot_row<WT>(u[t], xf));
-                        if (lane == 0) p.hrt[j] = silu_mul(a, b);
+                        if (lane == 0) p.hrt[j - (j % I) + hpos<WT>(j % I)] = silu_mul(a, b);
                     }
                 }
             }
@@ -357,7 +380,17 @@ __global__ void __launch_bounds__(D1_THREADS, 1) decode1_kernel(const __grid_con
 
         // ------------------------------------------------------------ phase C
         grid_barrier(p.ctl, nblocks, bar_idx++, to);
-        if (l + 1 == p.n_layers) grid_release(p.ctl, nblocks);  // the launch's last barrier
+        if (nrows > 0 && threadIdx.x == 0) {
+            // the routed and the shared h rows (written by every block before the barrier)
+            // into shared memory, two bulk copies
+            fence_proxy_async_global();
+            fence_proxy_async_smem();
+            mbar_arrive_expect_tx(hbar, uint32_t(4 * (k + 1) * I));
+            bulk_g2s(smem + S.hbuf, p.hrt, uint32_t(4 * k * I), hbar);
+            bulk_g2s(smem + S.hbuf + 4 * k * I, hsh, uint32_t(4 * I), hbar);
+        }
+        // the launch's last barrier: count the block out (after the h copies are on their way)
+        if (l + 1 == p.n_layers) grid_release(p.ctl, nblocks);
         if (l + 1 < p.n_layers && threadIdx.x < 32) {
             // L2 prefetch of the next layer's router rows and shared gate/up rows (the rows
             // this block streams first in that layer)
@@ -370,27 +403,18 @@ __global__ void __launch_bounds__(D1_THREADS, 1) decode1_kernel(const __grid_con
             }
         }
         if (nrows > 0) {
-            if (threadIdx.x == 0) {
-                // the routed and the shared h rows (written by every block before the
-                // barrier) into shared memory, two bulk copies
-                fence_proxy_async_global();
-                fence_proxy_async_smem();
-                mbar_arrive_expect_tx(hbar, uint32_t(4 * (k + 1) * I));
-                bulk_g2s(smem + S.hbuf, p.hrt, uint32_t(4 * k * I), hbar);
-                bulk_g2s(smem + S.hbuf + 4 * k * I, hsh, uint32_t(4 * I), hbar);
-            }
             mbar_wait(hbar, par, err, to);
-            const float wsh = __ldcg(sgate);
+            const float wsh = *s_wsh;
 #pragma unroll 1
             for (int m = 0; m < MU; ++m) {
                 const int unit = warp + D1_WARPS * m;
                 if (unit < 2 * (k + 1)) {
                     const int u = unit >> 1;
                     float hh[D1_HPL];
-                    const float4* hv = reinterpret_cast<const float4*>(hbuf + size_t(u) * I + lane * D1_HPL);
+                    const float4* hv = reinterpret_cast<const float4*>(hbuf + size_t(u) * I) + lane;
 #pragma unroll
                     for (int i = 0; i < D1_HPL / 4; ++i) {
-                        const float4 v = hv[i];
+                        const float4 v = hv[32 * i];
                         hh[4 * i] = v.x; hh[4 * i + 1] = v.y; hh[4 * i + 2] = v.z; hh[4 * i + 3] = v.w;
                     }
                     const float wr = __shfl_sync(FULL, sel_w, u < k ? u : 0);
