@@ -164,7 +164,13 @@ __device__ __forceinline__ float warp_sum(float v) {
 // ------------------------------------------------------------ grid barrier
 // Barrier across all blocks of a cooperative launch (every block is resident, so every
 // block eventually arrives). Barrier number b of a launch waits until the arrival counter
-// reaches (b + 1) * nblocks; arrivals are fire-and-forget reductions. grid_exit() must end
+// reaches (b + 1) * nblocks; arrivals are fire-and-forget reductions. Memory order comes
+// from the reductions and loads themselves, with no separate fence: the block's threads
+// meet at __syncthreads, then thread 0 arrives with a release (cumulative over the writes
+// the barrier made it observe); a waiter polls with acquire loads and then releases its
+// block (or warp) with __syncthreads (__syncwarp), which orders the block's later reads
+// after the other blocks' writes. A bulk copy that reads such data still needs
+// fence.proxy.async first. grid_exit() or grid_release() must end
 // the launch: its last block resets the counter for the next launch. The wait is bounded:
 // after `timeout_ns` (or once another block has recorded a timeout) the block records
 // ERRBIT_TIMEOUT and continues, so a fault can never hang the GPU; the host reads the
@@ -172,8 +178,7 @@ __device__ __forceinline__ float warp_sum(float v) {
 __device__ __forceinline__ void grid_barrier(Control* ctl, unsigned nblocks, unsigned index, uint64_t timeout_ns) {
     __syncthreads();
     if (threadIdx.x == 0) {
-        __threadfence();
-        asm volatile("red.relaxed.gpu.global.add.u32 [%0], 1;" :: "l"(&ctl->bar_count) : "memory");
+        asm volatile("red.release.gpu.global.add.u32 [%0], 1;" :: "l"(&ctl->bar_count) : "memory");
         const unsigned target = (index + 1u) * nblocks;
         if (ld_acquire_gpu(&ctl->bar_count) < target) {
             const uint64_t t0 = globaltimer_ns();
@@ -187,7 +192,6 @@ __device__ __forceinline__ void grid_barrier(Control* ctl, unsigned nblocks, uns
                 }
             }
         }
-        __threadfence();
     }
     __syncthreads();
 }
@@ -197,8 +201,7 @@ __device__ __forceinline__ void grid_barrier(Control* ctl, unsigned nblocks, uns
 __device__ __forceinline__ void grid_arrive(Control* ctl) {
     __syncthreads();
     if (threadIdx.x == 0) {
-        __threadfence();
-        asm volatile("red.relaxed.gpu.global.add.u32 [%0], 1;" :: "l"(&ctl->bar_count) : "memory");
+        asm volatile("red.release.gpu.global.add.u32 [%0], 1;" :: "l"(&ctl->bar_count) : "memory");
     }
 }
 __device__ __forceinline__ void grid_wait(Control* ctl, unsigned nblocks, unsigned index, uint64_t timeout_ns) {
@@ -216,7 +219,6 @@ __device__ __forceinline__ void grid_wait(Control* ctl, unsigned nblocks, unsign
                 }
             }
         }
-        __threadfence();
     }
     __syncthreads();
 }
@@ -239,7 +241,6 @@ __device__ __forceinline__ void grid_wait_warp(Control* ctl, unsigned nblocks, u
                 }
             }
         }
-        __threadfence();
     }
     __syncwarp();
 }

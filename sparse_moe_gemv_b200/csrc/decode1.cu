@@ -260,20 +260,22 @@ __global__ void __launch_bounds__(D1_THREADS, 1) decode1_kernel(const __grid_con
             const unsigned char* slot = dreg + u * S.slot;
 #pragma unroll
             for (int r = 0; r < D1_RB_MAX / 2; ++r) {
-                if (r < rn) {
+                {
+                    // rows past rn dot a valid row: no branch per row, the result is unused
+                    const int rr = min(ra + r, nrows - 1);
                     float2 d = make_float2(0.f, 0.f);
                     if constexpr (WT == DT_INT2) {
-                        const uint32_t wv = *reinterpret_cast<const uint32_t*>(slot + (ra + r) * drow + lane * 4);
-                        const float s = bf16f(*reinterpret_cast<const uint16_t*>(slot + S.sc_off + (ra + r) * dsc + (lane >> 1) * 2));
+                        const uint32_t wv = *reinterpret_cast<const uint32_t*>(slot + rr * drow + lane * 4);
+                        const float s = bf16f(*reinterpret_cast<const uint16_t*>(slot + S.sc_off + rr * dsc + (lane >> 1) * 2));
                         d = ffma2(make_float2(s, s), dot16_q2(wv, hf32), d);
                     } else if constexpr (WT == DT_INT4) {
-                        const uint2 wv = *reinterpret_cast<const uint2*>(slot + (ra + r) * drow + lane * 8);
-                        const float s = bf16f(*reinterpret_cast<const uint16_t*>(slot + S.sc_off + (ra + r) * dsc + (lane >> 1) * 2));
+                        const uint2 wv = *reinterpret_cast<const uint2*>(slot + rr * drow + lane * 8);
+                        const float s = bf16f(*reinterpret_cast<const uint16_t*>(slot + S.sc_off + rr * dsc + (lane >> 1) * 2));
                         const float2 a = dot8_q4(wv.x, hf32, make_float2(0.f, 0.f));
                         const float2 b = dot8_q4(wv.y, hf32 + 8, make_float2(0.f, 0.f));
                         d = ffma2(make_float2(s, s), fadd2(a, b), d);
                     } else {
-                        const unsigned char* wr = slot + (ra + r) * drow + lane * 16;
+                        const unsigned char* wr = slot + rr * drow + lane * 16;
                         const uint4 w0 = *reinterpret_cast<const uint4*>(wr);
                         const uint4 w1 = *reinterpret_cast<const uint4*>(wr + 512);
                         float2 e = make_float2(0.f, 0.f);
