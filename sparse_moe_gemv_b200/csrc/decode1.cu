@@ -48,25 +48,6 @@ namespace {
 
 __device__ __forceinline__ float hsum2(float2 v) { return warp_sum(v.x + v.y); }
 
-// Word of h element i (I = 512) in a staged h row. In phase C lane l holds the 16
-// elements its chunk of a down row covers: l*16 .. l*16+15 for int4 and int2 rows (one 8-
-// or 4-byte load), and l*8 .. l*8+7 with 256+l*8 .. 256+l*8+7 for bf16 rows (two 16-byte
-// loads 512 bytes apart, each conflict-free over the warp). Element m of lane l sits at
-// word 128*(m/4) + 4*l + m%4, so that the lane's four 16-byte loads of h are
-// conflict-free too.
-template <int WT>
-__device__ __forceinline__ int hpos(int i) {
-    int l, m;
-    if constexpr (WT == DT_BF16) {
-        l = (i & 255) >> 3;
-        m = (i & 7) | ((i >> 8) << 3);
-    } else {
-        l = i >> 4;
-        m = i & 15;
-    }
-    return 128 * (m >> 2) + 4 * l + (m & 3);
-}
-
 // Shared-memory plan of the kernel (byte offsets). `dreg` holds the block's rows of the
 // down matrix of k + 1 experts (routed slots 0..k-1 in selection order, the shared
 // expert in slot k), each slot RB rows (int4: codes, then scales).

@@ -221,7 +221,7 @@ __global__ void __launch_bounds__(D1_THREADS, 1) decodefr_kernel(const __grid_co
 #pragma unroll
                 for (int t = 0; t < T; ++t) {
                     const float av = hsum_fr(a[t]), bv = hsum_fr(b[t]);
-                    if (lane == 0) hsh[size_t(t) * I + i] = silu_mul(av, bv);
+                    if (lane == 0) hsh[size_t(t) * I + hpos<WT>(i)] = silu_mul(av, bv);
                 }
             }
         }
@@ -237,21 +237,23 @@ __global__ void __launch_bounds__(D1_THREADS, 1) decodefr_kernel(const __grid_co
 #pragma unroll
             for (int t = 0; t < T; ++t) {
                 if (mask >> t & 1u) {
-                    const float4* h4 = reinterpret_cast<const float4*>(hv[t] + lane * D1_HPL);
+                    const float4* h4 = reinterpret_cast<const float4*>(hv[t]) + lane;
 #pragma unroll
                     for (int i = 0; i < D1_HPL / 4; ++i) {
-                        const float4 v = h_global ? __ldcg(h4 + i) : h4[i];
+                        const float4 v = h_global ? __ldcg(h4 + 32 * i) : h4[32 * i];
                         hh[t][4 * i] = v.x; hh[t][4 * i + 1] = v.y; hh[t][4 * i + 2] = v.z; hh[t][4 * i + 3] = v.w;
                     }
                 }
             }
 #pragma unroll
             for (int r = 0; r < D1_RB_MAX / 2; ++r) {
-                if (r < rn) {
-                    const unsigned char* row = rows + (ra + r) * rstride;
+                {
+                    // rows past rn dot a valid row: no branch per row, the result is unused
+                    const int rr = min(ra + r, nrows - 1);
+                    const unsigned char* row = rows + rr * rstride;
                     if constexpr (WT == DT_INT4) {
                         const uint2 wv = *reinterpret_cast<const uint2*>(row + lane * 8);
-                        const float s = bf16f(*reinterpret_cast<const uint16_t*>(scl + (ra + r) * sstride + (lane >> 1) * 2));
+                        const float s = bf16f(*reinterpret_cast<const uint16_t*>(scl + rr * sstride + (lane >> 1) * 2));
 #pragma unroll
                         for (int t = 0; t < T; ++t) {
                             if (mask >> t & 1u) {
@@ -261,8 +263,8 @@ __global__ void __launch_bounds__(D1_THREADS, 1) decodefr_kernel(const __grid_co
                             }
                         }
                     } else {
-                        const uint4 w0 = *reinterpret_cast<const uint4*>(row + lane * 32);
-                        const uint4 w1 = *reinterpret_cast<const uint4*>(row + lane * 32 + 16);
+                        const uint4 w0 = *reinterpret_cast<const uint4*>(row + lane * 16);
+                        const uint4 w1 = *reinterpret_cast<const uint4*>(row + 512 + lane * 16);
                         const float2 f[8] = {bf2(w0.x), bf2(w0.y), bf2(w0.z), bf2(w0.w),
                                              bf2(w1.x), bf2(w1.y), bf2(w1.z), bf2(w1.w)};
 #pragma unroll
@@ -401,7 +403,7 @@ __global__ void __launch_bounds__(D1_THREADS, 1) decodefr_kernel(const __grid_co
                         for (int tt = 0; tt < T; ++tt) {
                             if (mask >> tt & 1u) {
                                 const float av = hsum_fr(a[tt]), bv = hsum_fr(b[tt]);
-                                if (lane == 0) p.hrt[size_t(s_us[uu * T + tt]) * I + i] = silu_mul(av, bv);
+                                if (lane == 0) p.hrt[size_t(s_us[uu * T + tt]) * I + hpos<WT>(i)] = silu_mul(av, bv);
                             }
                         }
                     }
@@ -409,7 +411,6 @@ __global__ void __launch_bounds__(D1_THREADS, 1) decodefr_kernel(const __grid_co
             }
         }
         grid_barrier(p.ctl, nblocks, bar_idx++, to);
-        if (l + 1 == p.n_layers) grid_release(p.ctl, nblocks);  // the launch's last barrier
 
         // ------------------------------------------------------------ phase C
         if (l + 1 < p.n_layers && threadIdx.x < 32) {
@@ -429,8 +430,10 @@ __global__ void __launch_bounds__(D1_THREADS, 1) decodefr_kernel(const __grid_co
                 mbar_arrive_expect_tx(hbar, uint32_t(4 * T * k * I));
                 bulk_g2s(smem + S.hbuf, p.hrt, uint32_t(4 * T * k * I), hbar);
             }
-            mbar_wait(hbar, par, err, to);
         }
+        // the launch's last barrier: count the block out (after the h copy is on its way)
+        if (l + 1 == p.n_layers) grid_release(p.ctl, nblocks);
+        if (nrows > 0) mbar_wait(hbar, par, err, to);
         float2 acc[D1_RB_MAX / 2][T];
 #pragma unroll
         for (int r = 0; r < D1_RB_MAX / 2; ++r)

@@ -176,6 +176,25 @@ __device__ __forceinline__ float2 dot_row_q2(const RowQ2& r, const float (&xf)[D
     return acc;
 }
 
+// Word of h element i (I = 512) in an h row as the down projection reads it. There lane l
+// holds the 16 elements its chunk of a down row covers: l*16 .. l*16+15 for int4 and int2
+// rows (one 8- or 4-byte load), and l*8 .. l*8+7 with 256+l*8 .. 256+l*8+7 for bf16 rows
+// (two 16-byte loads 512 bytes apart, each conflict-free over the warp). Element m of
+// lane l sits at word 128*(m/4) + 4*l + m%4, so that the lane's four 16-byte loads of h
+// are conflict-free (in shared memory) and coalesced (in global memory) too.
+template <int WT>
+__device__ __forceinline__ int hpos(int i) {
+    int l, m;
+    if constexpr (WT == DT_BF16) {
+        l = (i & 255) >> 3;
+        m = (i & 7) | ((i >> 8) << 3);
+    } else {
+        l = i >> 4;
+        m = i & 15;
+    }
+    return 128 * (m >> 2) + 4 * l + (m & 3);
+}
+
 template <int W> struct RowOf { using type = RowBF; };
 template <> struct RowOf<DT_INT4> { using type = RowQ4; };
 template <> struct RowOf<DT_INT2> { using type = RowQ2; };
