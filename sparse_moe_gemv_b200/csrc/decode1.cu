@@ -88,6 +88,29 @@ struct D1Params {
     DecLayer L[NL];
 };
 
+// x of one layer from pinned host memory into the workspace copy `xstage`, by warps 4..7
+// of one block (warps without a router row): each reads a quarter of x once over the link
+// with cache-volatile loads (the host rewrites it between calls), every load of a lane
+// issued before its first store so that the copy costs one link round trip, then counts
+// itself on x_ready with a release.
+__device__ __forceinline__ void fetch_host_x(const void* x, uint16_t* xstage, unsigned* x_ready, int H, int warp,
+                                             int lane) {
+    constexpr int PER = D1_XPL / 32;  // 16-byte chunks per lane: a quarter of x per warp
+    const uint4* src = static_cast<const uint4*>(x);
+    uint4* dst = reinterpret_cast<uint4*>(xstage);
+    const int c0 = (warp - 4) * 32 * PER + lane;
+    uint4 v[PER];
+#pragma unroll
+    for (int j = 0; j < PER; ++j)
+        if (c0 + 32 * j < H / 8) v[j] = __ldcv(src + c0 + 32 * j);
+#pragma unroll
+    for (int j = 0; j < PER; ++j)
+        if (c0 + 32 * j < H / 8) dst[c0 + 32 * j] = v[j];
+    __threadfence();
+    __syncwarp();
+    if (lane == 0) asm volatile("red.release.gpu.global.add.u32 [%0], 1;" :: "l"(x_ready) : "memory");
+}
+
 // XR: every layer's x comes from pinned host memory through p.xstage (a separate
 // instantiation, so that calls on device buffers carry none of that code).
 template <int WT, int NL, bool XR>
@@ -145,12 +168,12 @@ __global__ void __launch_bounds__(D1_THREADS, 1) decode1_kernel(const __grid_con
 
         // ------------------------------------------------------------ phase A
         constexpr bool xremote = XR;
-        if (xremote && blockIdx.x == 0 && warp >= 4) {
-            // x from host memory: warps 4..7 of block 0 (no router row) read it once over the
-            // link with cache-volatile loads (the host rewrites it between calls), every load
-            // of a lane issued before its first store so that the copy costs one link round
-            // trip, write it to the workspace and count themselves on x_ready
-            constexpr int PER = D1_XPL / 32;  // 16-byte chunks per lane: a quarter of x per warp
+        if (xremote && (NL == 1 || l == 0) && blockIdx.x == 0 && warp >= 4) {
+            // x from host memory, as fetch_host_x below: the first layer's is fetched by
+            // block 0 at the start of the launch, each later stacked layer's ahead of time
+            // (phase C); written out here rather than called, which keeps the single-layer
+            // build's registers as they were
+            constexpr int PER = D1_XPL / 32;
             const uint4* src = reinterpret_cast<const uint4*>(x);
             uint4* dst = reinterpret_cast<uint4*>(p.xstage);
             const int c0 = (warp - 4) * 32 * PER + lane;
@@ -363,6 +386,13 @@ __global__ void __launch_bounds__(D1_THREADS, 1) decode1_kernel(const __grid_con
 
         // ------------------------------------------------------------ phase C
         grid_barrier(p.ctl, nblocks, bar_idx++, to);
+        if constexpr (NL > 1) {
+            // the next stacked layer's x, fetched ahead by the last block (at the Qwen3-Next
+            // size it has no output rows, hence no phase-C work): every block copied this
+            // layer's staged x before the first barrier, so it may be overwritten now
+            if (XR && blockIdx.x == nblocks - 1 && warp >= 4 && l + 1 < p.n_layers)
+                fetch_host_x(p.L[l + 1].x, p.xstage, &p.ctl->x_ready, H, warp, lane);
+        }
         if (nrows > 0 && threadIdx.x == 0) {
             // the routed and the shared h rows (written by every block before the barrier)
             // into shared memory, two bulk copies
