@@ -87,6 +87,26 @@ struct FrParams {
     DecLayer L[NL];
 };
 
+// A quarter of one row of x (H/4 bf16 elements) from pinned host memory into the
+// workspace copy, by one warp: cache-volatile loads (the host rewrites x between calls),
+// every load of a lane issued before its first store (one link round trip), then a count
+// on x_ready with a release.
+__device__ __forceinline__ void fetch_host_quarter(const uint4* src_row, uint4* dst_row, int quarter, int H, int lane,
+                                                   unsigned* x_ready) {
+    constexpr int PER = D1_XPL / 32;  // 16-byte chunks per lane: a quarter row per warp
+    const int c0 = quarter * (H / 32) + lane;
+    uint4 v[PER];
+#pragma unroll
+    for (int j = 0; j < PER; ++j)
+        if (32 * j + lane < H / 32) v[j] = __ldcv(src_row + c0 + 32 * j);
+#pragma unroll
+    for (int j = 0; j < PER; ++j)
+        if (32 * j + lane < H / 32) dst_row[c0 + 32 * j] = v[j];
+    __threadfence();
+    __syncwarp();
+    if (lane == 0) asm volatile("red.release.gpu.global.add.u32 [%0], 1;" :: "l"(x_ready) : "memory");
+}
+
 // XR: x comes from pinned host memory through p.xstage (a separate instantiation, so
 // that calls on device buffers run without its waits and coherent loads).
 template <int WT, int T, int NL, bool XR>
@@ -151,10 +171,11 @@ __global__ void __launch_bounds__(D1_THREADS, 1) decodefr_kernel(const __grid_co
             issue_down(0, Ly.sh_down, Ly.sh_s_down);
         }
         bool xready = !xremote;  // this warp has seen the layer's x published
-        if (xremote && blockIdx.x < 4 * T && warp == D1_WARPS - 1) {
+        if (xremote && (NL == 1 || l == 0 || 4 * T > D1_WARPS) && blockIdx.x < 4 * T && warp == D1_WARPS - 1) {
             // x from host memory: a quarter of row blockIdx.x / 4 per block, read once over
             // the link with cache-volatile loads (the host rewrites it between calls), every
-            // load of a lane issued before its first store (one link round trip)
+            // load of a lane issued before its first store (one link round trip). A later
+            // stacked layer's x is fetched ahead, during the layer before (phase C).
             constexpr int PER = D1_XPL / 32;  // 16-byte chunks per lane: a quarter row per warp
             const uint4* src = static_cast<const uint4*>(Ly.x) + size_t(blockIdx.x >> 2) * (H / 8);
             uint4* dst = reinterpret_cast<uint4*>(p.xstage) + size_t(blockIdx.x >> 2) * (H / 8);
@@ -411,6 +432,15 @@ __global__ void __launch_bounds__(D1_THREADS, 1) decodefr_kernel(const __grid_co
             }
         }
         grid_barrier(p.ctl, nblocks, bar_idx++, to);
+        if constexpr (XR && NL > 1 && 4 * T <= D1_WARPS) {
+            // the next stacked layer's x, fetched ahead by the last block (at the Qwen3-Next
+            // size it has no output rows, hence no phase-C work), one quarter row per warp:
+            // every block's phase-B reads of this layer's staged x are behind the barrier
+            if (blockIdx.x == nblocks - 1 && warp < 4 * T && l + 1 < p.n_layers)
+                fetch_host_quarter(static_cast<const uint4*>(p.L[l + 1].x) + size_t(warp >> 2) * (H / 8),
+                                   reinterpret_cast<uint4*>(p.xstage) + size_t(warp >> 2) * (H / 8), warp & 3, H, lane,
+                                   &p.ctl->x_ready);
+        }
 
         // ------------------------------------------------------------ phase C
         if (l + 1 < p.n_layers && threadIdx.x < 32) {
