@@ -169,10 +169,10 @@ __global__ void __launch_bounds__(D1_THREADS, 1) decode1_kernel(const __grid_con
         // ------------------------------------------------------------ phase A
         constexpr bool xremote = XR;
         if (xremote && (NL == 1 || l == 0) && blockIdx.x == 0 && warp >= 4) {
-            // x from host memory, as fetch_host_x below: the first layer's is fetched by
-            // block 0 at the start of the launch, each later stacked layer's ahead of time
-            // (phase C); written out here rather than called, which keeps the single-layer
-            // build's registers as they were
+            // x from host memory, as in fetch_host_x: the first layer's is fetched by block 0
+            // at the start of the launch, each later stacked layer's ahead of time (phase
+            // C); written out here rather than called, which keeps the single-layer build's
+            // registers as they were
             constexpr int PER = D1_XPL / 32;
             const uint4* src = reinterpret_cast<const uint4*>(x);
             uint4* dst = reinterpret_cast<uint4*>(p.xstage);
